@@ -1,0 +1,174 @@
+"""Fused attention-distillation KL divergence for B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/streamkl.h`` (library
+``libstreamkl.so`` next to this file).  Every step of the computation runs in
+the library's CUDA kernels; this module only checks tensors, allocates outputs
+with torch and passes raw pointers.  There is no CPU fallback: if the library
+is missing or the device is not an sm_100 GPU, calls raise.
+
+Functions keep the C names:
+  streamkl_fwd(q_t, k_t, q_s, k_s, ...) -> (kl, lse_t, lse_s, loss_mean)
+  streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, ...) -> (dq_s, dk_s, dq_t, dk_t)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libstreamkl.so")
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "device wait timeout",
+          5: "workspace"}
+
+
+class StreamKLError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: run `python -m attention_kl_divergence_attn_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            shape = [_I] * 6 + [_F, _F, _I]
+            L.streamkl_fwd.argtypes = [_VP] * 4 + shape + [_VP] * 4 + [_VP, ctypes.c_size_t, _VP]
+            L.streamkl_fwd.restype = _I
+            L.streamkl_bwd.argtypes = ([_VP] * 4 + shape + [_VP] * 3 + [_VP, _F] + [_VP] * 4
+                                       + [_VP, ctypes.c_size_t, _VP])
+            L.streamkl_bwd.restype = _I
+            L.streamkl_workspace_size.argtypes = [_I] * 7
+            L.streamkl_workspace_size.restype = ctypes.c_size_t
+            L.streamkl_workspace_init.argtypes = [_VP, ctypes.c_size_t, _VP]
+            L.streamkl_workspace_init.restype = _I
+            L.streamkl_check.argtypes = [_VP, _VP, ctypes.POINTER(ctypes.c_uint)]
+            L.streamkl_check.restype = _I
+            L.streamkl_strerror.argtypes = [_I]
+            L.streamkl_strerror.restype = ctypes.c_char_p
+            L.streamkl_version.argtypes = []
+            L.streamkl_version.restype = _I
+            _lib = L
+    return _lib
+
+
+_workspaces: dict = {}
+
+
+def workspace(device=None) -> torch.Tensor:
+    """This device's workspace (status word), created and cleared on first use."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    ws = _workspaces.get(dev.index)
+    if ws is None:
+        n = lib().streamkl_workspace_size(0, 0, 0, 0, 0, 0, 0)
+        ws = torch.zeros(max(int(n), 16), dtype=torch.uint8, device=dev)
+        _workspaces[dev.index] = ws
+    return ws
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_inputs(q_t, k_t, q_s, k_s):
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("q_s", q_s), ("k_s", k_s)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
+    B, H, N_Q, d_t = q_t.shape
+    N_K = k_t.shape[2]
+    d_s = q_s.shape[3]
+    if k_t.shape != (B, H, N_K, d_t) or q_s.shape != (B, H, N_Q, d_s) or k_s.shape != (B, H, N_K, d_s):
+        raise ValueError("inconsistent shapes of q_t, k_t, q_s, k_s")
+    return B, H, N_Q, N_K, d_t, d_s
+
+
+def streamkl_fwd(q_t, k_t, q_s, k_s, scale_t=None, scale_s=None, causal=False, *, loss_mean=True,
+                 out=None, stream=None):
+    """Per-row KL(P_teacher || Q_student), both log-sum-exps and the mean loss.
+
+    Returns (kl, lse_t, lse_s, loss) with kl/lse_* fp32 [B, H, N_Q] and loss a
+    0-d fp32 device tensor (None if loss_mean=False).  ``out`` may supply the
+    three per-row buffers (and optionally a 4th, the loss scalar).
+    """
+    B, H, N_Q, N_K, d_t, d_s = _check_inputs(q_t, k_t, q_s, k_s)
+    scale_t = 1.0 / math.sqrt(d_t) if scale_t is None else float(scale_t)
+    scale_s = 1.0 / math.sqrt(d_s) if scale_s is None else float(scale_s)
+    dev = q_t.device
+    if out is None:
+        kl = torch.empty(B, H, N_Q, dtype=torch.float32, device=dev)
+        lse_t = torch.empty_like(kl)
+        lse_s = torch.empty_like(kl)
+        loss = torch.empty((), dtype=torch.float32, device=dev) if loss_mean else None
+    else:
+        kl, lse_t, lse_s = out[:3]
+        loss = (out[3] if len(out) > 3 else torch.empty((), dtype=torch.float32, device=dev)) if loss_mean else None
+    ws = workspace(dev)
+    rc = lib().streamkl_fwd(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
+                            scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
+                            _ptr(loss), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise StreamKLError("streamkl_fwd", rc)
+    return kl, lse_t, lse_s, loss
+
+
+def streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=None, causal=False, *,
+                 dkl=None, dloss=1.0, teacher_grads=False, out=None, stream=None):
+    """Gradients of sum_i g_i KL_i with g = dkl, or of dloss * mean(KL) if dkl is None.
+
+    Returns (dq_s, dk_s, dq_t, dk_t), fp32, the teacher pair None unless
+    teacher_grads.  ``out`` may supply the four buffers.
+    """
+    B, H, N_Q, N_K, d_t, d_s = _check_inputs(q_t, k_t, q_s, k_s)
+    scale_t = 1.0 / math.sqrt(d_t) if scale_t is None else float(scale_t)
+    scale_s = 1.0 / math.sqrt(d_s) if scale_s is None else float(scale_s)
+    for name, t in (("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s)) + ((("dkl", dkl),) if dkl is not None else ()):
+        if t.dtype != torch.float32 or t.numel() != B * H * N_Q or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 [B, H, N_Q] tensor")
+    dev = q_t.device
+    if out is None:
+        dq_s = torch.empty(B, H, N_Q, d_s, dtype=torch.float32, device=dev)
+        dk_s = torch.empty(B, H, N_K, d_s, dtype=torch.float32, device=dev)
+        dq_t = torch.empty(B, H, N_Q, d_t, dtype=torch.float32, device=dev) if teacher_grads else None
+        dk_t = torch.empty(B, H, N_K, d_t, dtype=torch.float32, device=dev) if teacher_grads else None
+    else:
+        dq_s, dk_s, dq_t, dk_t = out
+    ws = workspace(dev)
+    rc = lib().streamkl_bwd(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
+                            scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
+                            _ptr(dkl), float(dloss), _ptr(dq_s), _ptr(dk_s), _ptr(dq_t), _ptr(dk_t),
+                            _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise StreamKLError("streamkl_bwd", rc)
+    return dq_s, dk_s, dq_t, dk_t
+
+
+def streamkl_check(stream=None, device=None) -> int:
+    """Synchronises and raises if a kernel gave up on a bounded wait; returns the status word."""
+    ws = workspace(device)
+    code = ctypes.c_uint(0)
+    rc = lib().streamkl_check(_ptr(ws), _stream(stream), ctypes.byref(code))
+    if rc:
+        raise StreamKLError("streamkl_check", rc)
+    return code.value

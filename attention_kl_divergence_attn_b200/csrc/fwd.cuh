@@ -1,0 +1,279 @@
+// fwd.cuh — one-pass forward of the attention-distillation KL divergence.
+//
+// Source: "StreamKL: Fast and Memory-Efficient KL Divergence for Boosting
+// Attention Distillation", abstract — a single forward kernel that streams
+// query-key tiles through on-chip memory with an online formulation of the
+// coupled two-distribution KL reduction, so neither softmax is materialised.
+//
+// One CTA owns 128 query rows of one (batch, head).  Roles (6 warps):
+//   warp 0      TMA producer: Q_t, Q_s once; K_t, K_s tiles of 128 keys into
+//               an NSTAGE-deep shared-memory ring.
+//   warp 1      MMA issuer (one elected thread) and TMEM owner: per key tile
+//               S_t = Q_t K_t^T and S_s = Q_s K_s^T as tcgen05.mma (bf16 in,
+//               fp32 accumulate) into one of two TMEM buffers (2 x 256 cols).
+//   warps 2..5  softmax warpgroup: thread = query row = TMEM lane.  It reads
+//               its row of both logit tiles in 32-column chunks (tcgen05.ld
+//               32x32b), and updates the per-row online state
+//               (M_t, l_t, A, M_s, l_s); row reductions are thread-local
+//               because the 32x32b layout gives each thread one whole row.
+// State (log2 units, y = scale * log2(e) * q.k):
+//   M_t, M_s  running maxima of y_t, y_s
+//   l_t = sum 2^(y_t - M_t),  l_s = sum 2^(y_s - M_s)
+//   A   = sum 2^(y_t - M_t) (y_t - y_s)
+// and at the end LSE = ln2 (M + log2 l), KL = ln2 (A / l_t) - LSE_t + LSE_s.
+// Fully masked key tiles (above the causal diagonal) are never loaded.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace skl {
+
+struct FwdParams {
+    int BH, N_Q, N_K, causal, n_qt;
+    float ct, cs;          // scale_t * log2(e), scale_s * log2(e)
+    float *kl, *lse_t, *lse_s;
+    DevStatus st;
+};
+
+template <int DT, int DS>
+struct FwdCfg {
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int BLK = 128 * 128;                    // one [128 rows][64] bf16 box
+    static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
+    static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
+    static constexpr int Q_BYTES = QT_BYTES + QS_BYTES;
+    static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
+    static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
+    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
+    static constexpr int SMEM = Q_BYTES + NSTAGE * STAGE_BYTES + 1024;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+};
+
+// Number of key tiles a 128-row query tile starting at q0 must visit.
+__device__ __forceinline__ int fwd_key_tiles(int q0, int N_Q, int N_K, int causal, int BN) {
+    int kend = N_K;
+    if (causal) {
+        int last_row = min(q0 + 127, N_Q - 1);
+        kend = min(N_K, last_row + (N_K - N_Q) + 1);
+    }
+    return (kend + BN - 1) / BN;
+}
+
+// Online update with one 32-column chunk of raw logits (u = q.k, unscaled).
+template <bool MASKED>
+__device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
+                                             float &Ms, float &lt, float &ls, float &A) {
+    float m0 = fmaxf(ut[0], ut[1]), m1 = fmaxf(ut[2], ut[3]);
+    float n0 = fmaxf(us[0], us[1]), n1 = fmaxf(us[2], us[3]);
+#pragma unroll
+    for (int k = 4; k < 32; k += 4) {
+        m0 = fmaxf(m0, fmaxf(ut[k], ut[k + 1]));
+        m1 = fmaxf(m1, fmaxf(ut[k + 2], ut[k + 3]));
+        n0 = fmaxf(n0, fmaxf(us[k], us[k + 1]));
+        n1 = fmaxf(n1, fmaxf(us[k + 2], us[k + 3]));
+    }
+    const float Mt_new = fmaxf(Mt, fmaxf(m0, m1) * ct);
+    const float Ms_new = fmaxf(Ms, fmaxf(n0, n1) * cs);
+    if (MASKED && Mt_new == -INFINITY) return;      // nothing visible so far
+    const float at = ex2(Mt - Mt_new), as = ex2(Ms - Ms_new);
+    float st[4] = {0.f, 0.f, 0.f, 0.f}, ss[4] = {0.f, 0.f, 0.f, 0.f}, sa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float xt = fmaf(ut[k], ct, -Mt_new);
+        const float xs = fmaf(us[k], cs, -Ms_new);
+        const float et = ex2(xt), es = ex2(xs);
+        st[k & 3] += et;
+        ss[k & 3] += es;
+        float dx = xt - xs;
+        if (MASKED) dx = (ut[k] == -INFINITY) ? 0.f : dx;
+        sa[k & 3] = fmaf(et, dx, sa[k & 3]);
+    }
+    const float sum_t = (st[0] + st[1]) + (st[2] + st[3]);
+    const float sum_s = (ss[0] + ss[1]) + (ss[2] + ss[3]);
+    const float sum_a = (sa[0] + sa[1]) + (sa[2] + sa[3]);
+    lt = fmaf(lt, at, sum_t);
+    ls = fmaf(ls, as, sum_s);
+    A = fmaf(A, at, fmaf(Mt_new - Ms_new, sum_t, sum_a));
+    Mt = Mt_new;
+    Ms = Ms_new;
+}
+
+template <int DT, int DS>
+__global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
+    streamkl_fwd_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
+                        const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
+                        const FwdParams p) {
+    using C = FwdCfg<DT, DS>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQt = smem;
+    uint8_t *sQs = sQt + C::QT_BYTES;
+    uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
+
+    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_sempty[2];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // heaviest (latest) causal query tiles first
+    const int qt_idx = p.n_qt - 1 - (int)(blockIdx.x / p.BH);
+    const int bh = (int)(blockIdx.x % p.BH);
+    const int q0 = qt_idx * C::BM;
+    const int n_kt = fwd_key_tiles(q0, p.N_Q, p.N_K, p.causal, C::BN);
+    const int off = p.N_K - p.N_Q;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar_q, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(&bar_kfull[s], 1);
+            mbar_init(&bar_kempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar_sfull[b], 1);
+            mbar_init(&bar_sempty[b], 4);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int *abort_v = &abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (elect_one()) {
+            prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
+            mbar_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh);
+            int issued = 0;
+            for (int kt = 0; kt < n_kt; ++kt) {
+                const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
+                if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 1)) break;
+                uint8_t *st = sK + s * C::STAGE_BYTES;
+                mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
+#pragma unroll
+                for (int b = 0; b < DT / 64; ++b)
+                    tma_load_3d(st + b * C::BLK, &mKt, &bar_kfull[s], b * 64, kt * C::BN, bh);
+#pragma unroll
+                for (int b = 0; b < DS / 64; ++b)
+                    tma_load_3d(st + C::KT_BYTES + b * C::BLK, &mKs, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                issued = kt + 1;
+            }
+            if (*abort_v) {
+                // let copies already in flight land before the CTA's memory is released
+                DevStatus quick = p.st;
+                quick.budget_ns = 50000000ull;
+                volatile int never = 0;
+                for (int kt = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); kt < issued; ++kt)
+                    mbar_wait(&bar_kfull[kt % C::NSTAGE], (kt / C::NSTAGE) & 1, quick, &never, 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            if (mbar_wait(&bar_q, 0, p.st, abort_v, 2)) {
+                const uint32_t aQt = smem_u32(sQt), aQs = smem_u32(sQs);
+                for (int kt = 0; kt < n_kt; ++kt) {
+                    const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
+                    const int buf = kt & 1, use = kt >> 1;
+                    if (!mbar_wait(&bar_kfull[s], n & 1, p.st, abort_v, 3)) break;
+                    if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, p.st, abort_v, 4)) break;
+                    tc_fence_after();
+                    const uint32_t aKt = smem_u32(sK + s * C::STAGE_BYTES), aKs = aKt + C::KT_BYTES;
+                    const uint32_t dSt = tmem + buf * 256, dSs = dSt + 128;
+#pragma unroll
+                    for (int kk = 0; kk < DT / 16; ++kk) {
+                        const uint32_t o = (kk >> 2) * C::BLK + (kk & 3) * 32;
+                        mma_bf16_ss(dSt, sw128_desc(aQt + o, 16, 1024), sw128_desc(aKt + o, 16, 1024), C::IDESC,
+                                    kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < DS / 16; ++kk) {
+                        const uint32_t o = (kk >> 2) * C::BLK + (kk & 3) * 32;
+                        mma_bf16_ss(dSs, sw128_desc(aQs + o, 16, 1024), sw128_desc(aKs + o, 16, 1024), C::IDESC,
+                                    kk > 0);
+                    }
+                    mma_commit(&bar_sfull[buf]);
+                    mma_commit(&bar_kempty[s]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroup
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        const int grow = q0 + row;
+        const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
+        for (int kt = 0; kt < n_kt; ++kt) {
+            const int buf = kt & 1, use = kt >> 1;
+            if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 5)) break;
+            tc_fence_after();
+            const int k0 = kt * C::BN;
+            const bool masked = (k0 + C::BN > p.N_K) || (p.causal && (k0 + C::BN - 1 > q0 + off));
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float ut[32], us[32];
+                tmem_ld32(lane_base + buf * 256 + c * 32, ut);
+                tmem_ld32(lane_base + buf * 256 + 128 + c * 32, us);
+                tmem_ld_wait();
+                if (masked) {
+                    const int lim = p.causal ? min(p.N_K, grow + off + 1) : p.N_K;   // first hidden key
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        if (k0 + c * 32 + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }
+                    }
+                    online_chunk<true>(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                } else {
+                    online_chunk<false>(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_sempty[buf]);
+        }
+        if (grow < p.N_Q && !*abort_v) {
+            const float LN2 = 0.69314718055994530942f;
+            const float lse_t2 = Mt + lg2(lt), lse_s2 = Ms + lg2(ls);
+            const size_t r = (size_t)bh * p.N_Q + grow;
+            p.lse_t[r] = lse_t2 * LN2;
+            p.lse_s[r] = lse_s2 * LN2;
+            p.kl[r] = LN2 * (A / lt - lse_t2 + lse_s2);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Deterministic mean of n per-row values (one CTA, fp64 partial sums).
+__global__ void __launch_bounds__(1024) streamkl_mean_kernel(const float *__restrict__ v, long long n,
+                                                             float *__restrict__ out) {
+    __shared__ double red[1024];
+    double s = 0.0;
+    for (long long k = threadIdx.x; k < n; k += blockDim.x) s += (double)v[k];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *out = n > 0 ? (float)(red[0] / (double)n) : 0.f;
+}
+
+}  // namespace skl

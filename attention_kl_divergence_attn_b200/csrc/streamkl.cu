@@ -1,0 +1,188 @@
+// streamkl.cu — the C ABI declared in include/streamkl.h: argument checks,
+// TMA descriptor set-up and kernel launches.  No entry point allocates device
+// memory, synchronises (except streamkl_check) or aborts.
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "streamkl.h"
+#include "sm100.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+using namespace skl;
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;
+constexpr unsigned long long kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
+constexpr float kLog2e = 1.4426950408889634074f;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [BH, N, d] bf16 tensor: box = 64 columns x `rows` rows x 1
+// head, 128-byte swizzle, zero fill outside [0,N) so ragged tiles read zeros.
+bool make_map(CUtensorMap *m, const void *ptr, int d, int N, int BH, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+streamkl_status check_device() {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return STREAMKL_ERR_CUDA;
+    return major == 10 ? STREAMKL_OK : STREAMKL_ERR_UNSUPPORTED;
+}
+
+streamkl_status check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal, float scale_t,
+                            float scale_s) {
+    if (B < 0 || H < 0 || N_Q < 0 || N_K < 0) return STREAMKL_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return STREAMKL_ERR_INVALID_ARG;
+    if (causal && N_Q > N_K) return STREAMKL_ERR_INVALID_ARG;
+    if (!causal && N_K == 0 && N_Q > 0 && B > 0 && H > 0) return STREAMKL_ERR_INVALID_ARG;
+    if (!(scale_t > 0.f) || !(scale_s > 0.f) || scale_t == INFINITY || scale_s == INFINITY)
+        return STREAMKL_ERR_INVALID_ARG;
+    if ((long long)B * H > (1ll << 24) || N_Q > (1 << 24) || N_K > (1 << 24)) return STREAMKL_ERR_INVALID_ARG;
+    if ((d_t != 64 && d_t != 128) || (d_s != 64 && d_s != 128)) return STREAMKL_ERR_UNSUPPORTED;
+    return STREAMKL_OK;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int DT, int DS>
+streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const CUtensorMap &qs,
+                           const CUtensorMap &ks, const FwdParams &p, cudaStream_t stream) {
+    using C = FwdCfg<DT, DS>;
+    auto kern = streamkl_fwd_kernel<DT, DS>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    const long long grid = (long long)p.BH * p.n_qt;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
+    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int streamkl_version(void) { return 100; }
+
+size_t streamkl_workspace_size(int, int, int, int, int, int, int) { return kWorkspaceBytes; }
+
+const char *streamkl_strerror(streamkl_status s) {
+    switch (s) {
+        case STREAMKL_OK: return "ok";
+        case STREAMKL_ERR_INVALID_ARG: return "invalid argument";
+        case STREAMKL_ERR_UNSUPPORTED: return "unsupported problem or device";
+        case STREAMKL_ERR_CUDA: return "CUDA error";
+        case STREAMKL_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+        case STREAMKL_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+    if (!workspace) return STREAMKL_ERR_WORKSPACE;
+    if (workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
+    return cudaMemsetAsync(workspace, 0, kWorkspaceBytes, (cudaStream_t)stream) == cudaSuccess ? STREAMKL_OK
+                                                                                             : STREAMKL_ERR_CUDA;
+}
+
+streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int *code_out) {
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    unsigned int word = 0;
+    if (workspace) {
+        if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return STREAMKL_ERR_CUDA;
+        if (cudaMemsetAsync(const_cast<void *>(workspace), 0, sizeof word, s) != cudaSuccess)
+            return STREAMKL_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    if (code_out) *code_out = word;
+    if (cudaPeekAtLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    return (word & kStatusTimeout) ? STREAMKL_ERR_TIMEOUT : STREAMKL_OK;
+}
+
+streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                             int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
+                             float *kl, float *lse_t, float *lse_s, float *loss_mean, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
+    if (st != STREAMKL_OK) return st;
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int BH = B * H;
+    const long long rows = (long long)BH * N_Q;
+    if (rows == 0) {
+        if (loss_mean) streamkl_mean_kernel<<<1, 1024, 0, s>>>(kl, 0, loss_mean);
+        return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+    }
+    if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s)) return STREAMKL_ERR_INVALID_ARG;
+    if ((st = check_device()) != STREAMKL_OK) return st;
+
+    CUtensorMap mqt, mkt, mqs, mks;
+    if (!make_map(&mqt, q_t, d_t, N_Q, BH, 128) || !make_map(&mkt, k_t, d_t, N_K, BH, 128) ||
+        !make_map(&mqs, q_s, d_s, N_Q, BH, 128) || !make_map(&mks, k_s, d_s, N_K, BH, 128))
+        return STREAMKL_ERR_CUDA;
+    FwdParams p;
+    p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
+    p.n_qt = (N_Q + 127) / 128;
+    p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
+    p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s;
+    p.st.word = static_cast<uint32_t *>(workspace);
+    p.st.budget_ns = kWaitBudgetNs;
+    if (d_t == 64 && d_s == 64) st = launch_fwd<64, 64>(mqt, mkt, mqs, mks, p, s);
+    else if (d_t == 128 && d_s == 128) st = launch_fwd<128, 128>(mqt, mkt, mqs, mks, p, s);
+    else if (d_t == 128 && d_s == 64) st = launch_fwd<128, 64>(mqt, mkt, mqs, mks, p, s);
+    else st = launch_fwd<64, 128>(mqt, mkt, mqs, mks, p, s);
+    if (st != STREAMKL_OK) return st;
+    if (loss_mean) {
+        streamkl_mean_kernel<<<1, 1024, 0, s>>>(kl, rows, loss_mean);
+        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    return STREAMKL_OK;
+}
+
+}  // extern "C"
+
+extern "C" streamkl_status streamkl_bwd(const void *, const void *, const void *, const void *, int, int, int, int,
+                                        int, int, float, float, int, const float *, const float *, const float *,
+                                        const float *, float, float *, float *, float *, float *, void *, size_t,
+                                        void *) {
+    return STREAMKL_ERR_UNSUPPORTED;
+}

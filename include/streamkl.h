@@ -1,0 +1,124 @@
+/*
+ * streamkl.h — C ABI of the fused attention-distillation KL divergence on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation ("StreamKL: Fast and Memory-Efficient KL Divergence for
+ * Boosting Attention Distillation", abstract): one attention distribution,
+ * the teacher P = softmax(scale_t * Q_t K_t^T), is compared with another, the
+ * student Q = softmax(scale_s * Q_s K_s^T), row by row through their KL
+ * divergence KL_i = sum_j P_ij (log P_ij - log Q_ij) (teacher in the first
+ * slot, "Lecture 05 - Where It All Lands ...", section 3.1), and the loss is
+ * the mean of KL_i over every (batch, head, query row).  The forward is one
+ * pass over key tiles held on chip, keeping an online per-row state for both
+ * distributions; the backward recomputes both distributions tile by tile from
+ * the saved per-row log-sum-exps.  Neither pass writes an N_Q x N_K buffer,
+ * and the library never allocates device memory: every buffer is the
+ * caller's.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are dense row-major with the head dimension innermost:
+ *      Q_t [B, H, N_Q, d_t]   K_t [B, H, N_K, d_t]     (teacher, bf16)
+ *      Q_s [B, H, N_Q, d_s]   K_s [B, H, N_K, d_s]     (student, bf16)
+ *    per-row vectors are fp32 [B, H, N_Q]; gradients are fp32 and shaped like
+ *    the tensor they belong to.
+ *  - Every pointer is a DEVICE pointer on the current CUDA device, 16-byte
+ *    aligned, unless stated otherwise.  Inputs are read only.
+ *  - d_t and d_s must each be 64 or 128 (other sizes: STREAMKL_ERR_UNSUPPORTED).
+ *    N_Q, N_K need not be multiples of any tile size.
+ *  - causal: key j is visible to query i iff j <= i + (N_K - N_Q) (the mask's
+ *    diagonal ends at the bottom-right corner); causal with N_Q > N_K is
+ *    rejected (rows without a visible key).  Non-causal needs N_K >= 1.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous: a return of STREAMKL_OK means the launch was
+ *    accepted.  Errors found on the device (a bounded wait that gave up) are
+ *    recorded in the caller's workspace and reported by streamkl_check().
+ *  - `workspace` is device memory of at least streamkl_workspace_size() bytes,
+ *    owned by the caller, cleared once with streamkl_workspace_init() before
+ *    first use.  It holds a sticky device status word that kernels set when a
+ *    bounded wait gives up; streamkl_check() reads and clears it.  Calls that
+ *    share one workspace may overlap on the GPU (the word is only OR-ed).
+ *  - No entry point aborts, prints, or allocates; on an argument error nothing
+ *    is launched.
+ */
+#ifndef STREAMKL_H
+#define STREAMKL_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STREAMKL_OK = 0,
+    STREAMKL_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape or flag */
+    STREAMKL_ERR_UNSUPPORTED = 2,   /* valid problem the kernels do not cover (d not 64/128, no sm_100 device) */
+    STREAMKL_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+    STREAMKL_ERR_TIMEOUT = 4,       /* a kernel gave up on a bounded wait (see streamkl_check) */
+    STREAMKL_ERR_WORKSPACE = 5      /* workspace NULL or smaller than streamkl_workspace_size() */
+} streamkl_status;
+
+/* Bytes of device workspace a call needs for this problem (a small constant:
+ * the device status word; nothing grows with N_Q or N_K). */
+size_t streamkl_workspace_size(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal);
+
+/*
+ * Forward.  For every (b, h, i) writes
+ *   lse_t[b,h,i] = log sum_j exp(scale_t <Q_t[i], K_t[j]>)   (visible j, natural log)
+ *   lse_s[b,h,i] = the same for the student
+ *   kl[b,h,i]    = sum_j P_ij (log P_ij - log Q_ij)           (nats, not clamped)
+ * and, if loss_mean != NULL, the device scalar loss_mean = mean over all
+ * B*H*N_Q rows of kl (a deterministic reduction).
+ * Source: the abstract's single one-pass forward kernel with the online
+ * formulation of the coupled two-distribution KL reduction.
+ * kl, lse_t, lse_s: required, fp32 [B,H,N_Q].  They are what streamkl_bwd needs.
+ */
+streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                             int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                             float scale_t, float scale_s, int causal,
+                             float *kl, float *lse_t, float *lse_s, float *loss_mean,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Backward.  With the upstream gradient g_i = dL/dKL_i taken from `dkl`
+ * ([B,H,N_Q] fp32) or, when dkl == NULL, g_i = dloss / (B*H*N_Q) (the
+ * gradient of loss_mean scaled by dloss), writes
+ *   dq_s = dL/dQ_s, dk_s = dL/dK_s                (always; fp32)
+ *   dq_t = dL/dQ_t, dk_t = dL/dK_t                (only if both are non-NULL)
+ * where, per visible (i, j),
+ *   dS_s = g_i (Q_ij - P_ij),  dS_t = g_i P_ij (log P_ij - log Q_ij - KL_i),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q   (teacher side with scale_t).
+ * Source: the abstract's backward, which recomputes the attention
+ * probabilities tile by tile instead of storing quadratic intermediates.
+ * kl, lse_t, lse_s must be the outputs of streamkl_fwd on the same inputs.
+ * Gradient outputs are overwritten (not accumulated).  dq_t and dk_t must be
+ * both NULL (student gradients only) or both non-NULL.
+ */
+streamkl_status streamkl_bwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                             int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                             float scale_t, float scale_s, int causal,
+                             const float *kl, const float *lse_t, const float *lse_s,
+                             const float *dkl, float dloss,
+                             float *dq_s, float *dk_s, float *dq_t, float *dk_t,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Clears the workspace (enqueued on `stream`).  Needed once per workspace. */
+streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream` and returns STREAMKL_ERR_TIMEOUT if a kernel of an
+ * earlier call on this workspace gave up on a bounded wait, STREAMKL_ERR_CUDA
+ * if the stream reports a CUDA error, else STREAMKL_OK.  `code_out` (host
+ * pointer, nullable) receives the raw device status word (0 = clean). */
+streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int *code_out);
+
+/* Static, human-readable name of a status. */
+const char *streamkl_strerror(streamkl_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int streamkl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMKL_H */
