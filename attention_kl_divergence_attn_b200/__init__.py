@@ -53,6 +53,13 @@ def lib():
             L.streamkl_bwd.argtypes = ([_VP] * 4 + shape + [_VP] * 3 + [_VP, _F] + [_VP] * 4
                                        + [_VP, ctypes.c_size_t, _VP])
             L.streamkl_bwd.restype = _I
+            L.streamkl_bwd_dk.argtypes = ([_VP] * 4 + shape + [_VP] * 3 + [_VP, _F] + [_VP] * 2
+                                          + [_VP, ctypes.c_size_t, _VP])
+            L.streamkl_bwd_dk.restype = _I
+            L.streamkl_bwd_dq.argtypes = L.streamkl_bwd_dk.argtypes
+            L.streamkl_bwd_dq.restype = _I
+            L.streamkl_loss_mean.argtypes = [_VP, ctypes.c_longlong, _VP, _VP]
+            L.streamkl_loss_mean.restype = _I
             L.streamkl_workspace_size.argtypes = [_I] * 7
             L.streamkl_workspace_size.restype = ctypes.c_size_t
             L.streamkl_workspace_init.argtypes = [_VP, ctypes.c_size_t, _VP]
@@ -162,6 +169,52 @@ def streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=Non
     if rc:
         raise StreamKLError("streamkl_bwd", rc)
     return dq_s, dk_s, dq_t, dk_t
+
+
+def _bwd_part(fn, which, q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s, causal, dkl, dloss,
+              teacher_grads, out, stream):
+    B, H, N_Q, N_K, d_t, d_s = _check_inputs(q_t, k_t, q_s, k_s)
+    scale_t = 1.0 / math.sqrt(d_t) if scale_t is None else float(scale_t)
+    scale_s = 1.0 / math.sqrt(d_s) if scale_s is None else float(scale_s)
+    dev = q_t.device
+    n = N_K if which == "k" else N_Q
+    if out is None:
+        g_s = torch.empty(B, H, n, d_s, dtype=torch.float32, device=dev)
+        g_t = torch.empty(B, H, n, d_t, dtype=torch.float32, device=dev) if teacher_grads else None
+    else:
+        g_s, g_t = out
+    ws = workspace(dev)
+    rc = getattr(lib(), fn)(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
+                            scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
+                            _ptr(dkl), float(dloss), _ptr(g_s), _ptr(g_t), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise StreamKLError(fn, rc)
+    return g_s, g_t
+
+
+def streamkl_bwd_dk(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=None, causal=False, *,
+                    dkl=None, dloss=1.0, teacher_grads=False, out=None, stream=None):
+    """Key gradients only: (dk_s, dk_t), the teacher one None unless teacher_grads."""
+    return _bwd_part("streamkl_bwd_dk", "k", q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s, causal,
+                     dkl, dloss, teacher_grads, out, stream)
+
+
+def streamkl_bwd_dq(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=None, causal=False, *,
+                    dkl=None, dloss=1.0, teacher_grads=False, out=None, stream=None):
+    """Query gradients only: (dq_s, dq_t), the teacher one None unless teacher_grads."""
+    return _bwd_part("streamkl_bwd_dq", "q", q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s, causal,
+                     dkl, dloss, teacher_grads, out, stream)
+
+
+def streamkl_loss_mean(kl, out=None, stream=None):
+    """Deterministic mean of a contiguous fp32 per-row KL tensor, as a 0-d device tensor."""
+    if kl.dtype != torch.float32 or not kl.is_cuda or not kl.is_contiguous():
+        raise TypeError("kl must be a contiguous CUDA fp32 tensor")
+    out = torch.empty((), dtype=torch.float32, device=kl.device) if out is None else out
+    rc = lib().streamkl_loss_mean(_ptr(kl), kl.numel(), _ptr(out), _stream(stream))
+    if rc:
+        raise StreamKLError("streamkl_loss_mean", rc)
+    return out
 
 
 def streamkl_check(stream=None, device=None) -> int:

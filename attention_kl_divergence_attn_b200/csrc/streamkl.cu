@@ -93,40 +93,99 @@ streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const C
     return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
+// Which backward kernels a call launches.
+enum BwdParts { kPartDK = 1, kPartDQ = 2 };
+
 template <int DT, int DS, bool TEACHER>
 streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int N_Q, int N_K,
-                           BwdParams p, cudaStream_t stream) {
+                           BwdParams p, int parts, cudaStream_t stream) {
     using CK = DkvCfg<DT, DS, TEACHER>;
     using CQ = DqCfg<DT, DS, TEACHER>;
     const int BH = p.BH;
-    // key-owner kernel: K boxes of 128 rows, Q boxes of 64 rows
     CUtensorMap mqt, mkt, mqs, mks;
-    if (!make_map(&mqt, q_t, DT, N_Q, BH, CK::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CK::BN) ||
-        !make_map(&mqs, q_s, DS, N_Q, BH, CK::BM) || !make_map(&mks, k_s, DS, N_K, BH, CK::BN))
-        return STREAMKL_ERR_CUDA;
-    auto kdkv = streamkl_bwd_dkv_kernel<DT, DS, TEACHER>;
-    if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
-    p.n_tiles = (N_K + CK::BN - 1) / CK::BN;
-    kdkv<<<(unsigned)((long long)BH * p.n_tiles), CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
-    if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
-    // query-owner kernel: Q boxes of 128 rows, K boxes of 64 rows
-    if (!make_map(&mqt, q_t, DT, N_Q, BH, CQ::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CQ::BN) ||
-        !make_map(&mqs, q_s, DS, N_Q, BH, CQ::BM) || !make_map(&mks, k_s, DS, N_K, BH, CQ::BN))
-        return STREAMKL_ERR_CUDA;
-    auto kdq = streamkl_bwd_dq_kernel<DT, DS, TEACHER>;
-    if (set_smem(kdq, CQ::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
-    p.n_tiles = (N_Q + CQ::BM - 1) / CQ::BM;
-    kdq<<<(unsigned)((long long)BH * p.n_tiles), CQ::THREADS, CQ::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
-    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+    if (parts & kPartDK) {
+        // key-owner kernel: K boxes of 128 rows, Q boxes of 64 rows
+        if (!make_map(&mqt, q_t, DT, N_Q, BH, CK::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CK::BN) ||
+            !make_map(&mqs, q_s, DS, N_Q, BH, CK::BM) || !make_map(&mks, k_s, DS, N_K, BH, CK::BN))
+            return STREAMKL_ERR_CUDA;
+        auto kdkv = streamkl_bwd_dkv_kernel<DT, DS, TEACHER>;
+        if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+        p.n_tiles = (N_K + CK::BN - 1) / CK::BN;
+        kdkv<<<(unsigned)((long long)BH * p.n_tiles), CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    if (parts & kPartDQ) {
+        // query-owner kernel: Q boxes of 128 rows, K boxes of 64 rows
+        if (!make_map(&mqt, q_t, DT, N_Q, BH, CQ::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CQ::BN) ||
+            !make_map(&mqs, q_s, DS, N_Q, BH, CQ::BM) || !make_map(&mks, k_s, DS, N_K, BH, CQ::BN))
+            return STREAMKL_ERR_CUDA;
+        auto kdq = streamkl_bwd_dq_kernel<DT, DS, TEACHER>;
+        if (set_smem(kdq, CQ::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+        p.n_tiles = (N_Q + CQ::BM - 1) / CQ::BM;
+        kdq<<<(unsigned)((long long)BH * p.n_tiles), CQ::THREADS, CQ::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    return STREAMKL_OK;
 }
 
 template <bool TEACHER>
 streamkl_status dispatch_bwd(int d_t, int d_s, const void *q_t, const void *k_t, const void *q_s, const void *k_s,
-                             int N_Q, int N_K, const BwdParams &p, cudaStream_t s) {
-    if (d_t == 64 && d_s == 64) return launch_bwd<64, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, s);
-    if (d_t == 128 && d_s == 128) return launch_bwd<128, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, s);
-    if (d_t == 128 && d_s == 64) return launch_bwd<128, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, s);
-    return launch_bwd<64, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, s);
+                             int N_Q, int N_K, const BwdParams &p, int parts, cudaStream_t s) {
+    if (d_t == 64 && d_s == 64) return launch_bwd<64, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+    if (d_t == 128 && d_s == 128) return launch_bwd<128, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+    if (d_t == 128 && d_s == 64) return launch_bwd<128, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+    return launch_bwd<64, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+}
+
+// Shared body of the three backward entry points.  `parts` selects the
+// kernels; the gradient pointers a part does not write may be NULL.
+streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                           int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
+                           const float *kl, const float *lse_t, const float *lse_s, const float *dkl, float dloss,
+                           float *dq_s, float *dk_s, float *dq_t, float *dk_t, void *workspace,
+                           size_t workspace_bytes, void *stream, int parts) {
+    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
+    if (st != STREAMKL_OK) return st;
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
+    const bool want_dk = parts & kPartDK, want_dq = parts & kPartDQ;
+    // the teacher pair of each part must be both given or both absent
+    if (want_dk && want_dq && ((dq_t == nullptr) != (dk_t == nullptr))) return STREAMKL_ERR_INVALID_ARG;
+    const bool teacher = want_dk ? dk_t != nullptr : dq_t != nullptr;
+    if (!(dloss == dloss)) return STREAMKL_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int BH = B * H;
+    if (want_dk && (!dk_s || (teacher && !dk_t))) return STREAMKL_ERR_INVALID_ARG;
+    if (want_dq && (!dq_s || (teacher && !dq_t))) return STREAMKL_ERR_INVALID_ARG;
+    if ((long long)BH * N_K == 0) return STREAMKL_OK;       // no keys (so no rows either): nothing to write
+    if ((long long)BH * N_Q == 0) {                         // keys but no queries: every dK is zero
+        if (want_dk) {
+            if (cudaMemsetAsync(dk_s, 0, (size_t)BH * N_K * d_s * sizeof(float), s) != cudaSuccess)
+                return STREAMKL_ERR_CUDA;
+            if (teacher && cudaMemsetAsync(dk_t, 0, (size_t)BH * N_K * d_t * sizeof(float), s) != cudaSuccess)
+                return STREAMKL_ERR_CUDA;
+        }
+        return STREAMKL_OK;
+    }
+    if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s)) return STREAMKL_ERR_INVALID_ARG;
+    if (want_dk && (!aligned16(dk_s) || (teacher && !aligned16(dk_t)))) return STREAMKL_ERR_INVALID_ARG;
+    if (want_dq && (!aligned16(dq_s) || (teacher && !aligned16(dq_t)))) return STREAMKL_ERR_INVALID_ARG;
+    if ((st = check_device()) != STREAMKL_OK) return st;
+
+    BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
+    p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
+    p.out_t = scale_t * 0.69314718055994530942f;
+    p.out_s = scale_s;
+    p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s; p.dkl = dkl;
+    p.g_const = (float)((double)dloss / ((double)BH * (double)N_Q));
+    p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
+    p.st.word = static_cast<uint32_t *>(workspace);
+    p.st.budget_ns = kWaitBudgetNs;
+    return teacher ? dispatch_bwd<true>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s)
+                   : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
 }
 
 }  // namespace
@@ -221,42 +280,32 @@ streamkl_status streamkl_bwd(const void *q_t, const void *k_t, const void *q_s, 
                              const float *kl, const float *lse_t, const float *lse_s, const float *dkl, float dloss,
                              float *dq_s, float *dk_s, float *dq_t, float *dk_t, void *workspace,
                              size_t workspace_bytes, void *stream) {
-    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
-    if (st != STREAMKL_OK) return st;
-    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
-    if ((dq_t == nullptr) != (dk_t == nullptr)) return STREAMKL_ERR_INVALID_ARG;
-    if (!(dloss == dloss)) return STREAMKL_ERR_INVALID_ARG;
-    const bool teacher = dq_t != nullptr;
-    cudaStream_t s = (cudaStream_t)stream;
-    const int BH = B * H;
-    if ((long long)BH * N_K == 0) return STREAMKL_OK;       // no keys (so no rows either): nothing to write
-    if (!dk_s || (teacher && !dk_t)) return STREAMKL_ERR_INVALID_ARG;
-    if ((long long)BH * N_Q == 0) {                         // keys but no queries: every dK is zero
-        if (cudaMemsetAsync(dk_s, 0, (size_t)BH * N_K * d_s * sizeof(float), s) != cudaSuccess) return STREAMKL_ERR_CUDA;
-        if (teacher && cudaMemsetAsync(dk_t, 0, (size_t)BH * N_K * d_t * sizeof(float), s) != cudaSuccess)
-            return STREAMKL_ERR_CUDA;
-        return STREAMKL_OK;
-    }
-    if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s || !dq_s) return STREAMKL_ERR_INVALID_ARG;
-    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s) || !aligned16(dq_s) ||
-        !aligned16(dk_s) || (teacher && (!aligned16(dq_t) || !aligned16(dk_t))))
-        return STREAMKL_ERR_INVALID_ARG;
-    if ((st = check_device()) != STREAMKL_OK) return st;
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+                      dloss, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes, stream, kPartDK | kPartDQ);
+}
 
-    BwdParams p;
-    memset(&p, 0, sizeof p);
-    p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
-    p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
-    p.out_t = scale_t * 0.69314718055994530942f;
-    p.out_s = scale_s;
-    p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s; p.dkl = dkl;
-    p.g_const = (float)((double)dloss / ((double)BH * (double)N_Q));
-    p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
-    p.st.word = static_cast<uint32_t *>(workspace);
-    p.st.budget_ns = kWaitBudgetNs;
-    return teacher ? dispatch_bwd<true>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, s)
-                   : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, s);
+streamkl_status streamkl_bwd_dk(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                                int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
+                                const float *kl, const float *lse_t, const float *lse_s, const float *dkl,
+                                float dloss, float *dk_s, float *dk_t, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+                      dloss, nullptr, dk_s, nullptr, dk_t, workspace, workspace_bytes, stream, kPartDK);
+}
+
+streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                                int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
+                                const float *kl, const float *lse_t, const float *lse_s, const float *dkl,
+                                float dloss, float *dq_s, float *dq_t, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+                      dloss, dq_s, nullptr, dq_t, nullptr, workspace, workspace_bytes, stream, kPartDQ);
+}
+
+streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream) {
+    if (n_rows < 0 || !loss_mean || (n_rows > 0 && !kl)) return STREAMKL_ERR_INVALID_ARG;
+    streamkl_mean_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(kl, n_rows, loss_mean);
+    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention-distillation KL divergence (forward + backward).
+
+One step = the whole hot path on one batch: forward (per-row KL and both
+log-sum-exps), the mean loss, and the backward for every requested gradient
+(student dQ_s, dK_s and, for the headline workload, teacher dQ_t, dK_t).
+
+Default workload: B=1, H=32, N_Q=N_K=8192, d_t=d_s=128, causal, teacher and
+student Q/K drawn independently from N(0,1) in bf16, gradients of the mean
+loss for both teacher and student.  Throughput counts 2*N_Q*N_K*(d_t+d_s)
+forward FLOPs and 2*N_Q*N_K*(d_t+d_s) + 4*N_Q*N_K*(d_s + d_t) backward FLOPs
+per head, halved for causal masks (2.199 TFLOP per step here).
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
+  python bench.py --impl reference ...    # the fp64 CPU oracle on the same workload
+
+With N > 1 (torchrun, one process per GPU) every rank solves its own
+independent problem of the default size (heads are independent: no data-path
+collective); the value is the total FLOPs of all ranks over the slowest rank's
+device time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn-KL fwd+bwd TFLOP/s and % of B200 bf16 tensor peak (N=8192, d=128, causal)"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 2**20
+
+
+# ----------------------------------------------------------------------------- flop accounting
+
+def visible_pairs(w) -> float:
+    """Number of (query, key) pairs per head, the causal mask counted as a half."""
+    return w.N_Q * w.N_K / (2.0 if w.causal else 1.0)
+
+
+def step_flops(w) -> float:
+    per = 2 * (w.d_t + w.d_s) + 2 * (w.d_t + w.d_s) + 4 * w.d_s + (4 * w.d_t if w.teacher_grads else 0)
+    return per * visible_pairs(w) * w.B * w.H
+
+
+def kernel_flops(w) -> dict:
+    """MMA FLOPs each kernel issues per launch (what its tensor pipe executes)."""
+    n = visible_pairs(w) * w.B * w.H
+    s = 2 * (w.d_t + w.d_s)                      # S_t and S_s
+    g = 2 * w.d_s + (2 * w.d_t if w.teacher_grads else 0)
+    return {"streamkl_fwd_kernel": s * n, "streamkl_bwd_dkv_kernel": (s + g) * n,
+            "streamkl_bwd_dq_kernel": (s + g) * n, "streamkl_mean_kernel": 0.0}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling of one GPU while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self) -> dict:
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, pw, reasons = [], None, [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                pw.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s, p in zip(sm, pw) if p > 250.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(loaded), "power_w_max": max(pw)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_kl_divergence_attn_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary of the current sources, else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    e = rec.get("kernels", {}).get(kernel, {})
+    if e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, n_rows: int, seed: int, cores: int):
+    """Times the fp64 oracle on `n_rows` seeded rows of head (0, 0): forward of
+    those rows plus their full backward (dQ rows and dK contributions).
+    Returns (seconds, metric FLOPs of the sampled (query, key) pairs)."""
+    import numpy as np
+    import oracle
+    from attention_kl_divergence_attn_b200 import inputs
+    qt, kt, qs, ks = (t[None, None] for t in inputs.head_inputs(w, 0, 0))
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.N_Q, size=min(n_rows, w.N_Q), replace=False)).astype(np.int64)
+    qt, kt, qs, ks = (oracle._f64(x) for x in (qt, kt, qs, ks))
+    g = 1.0 / w.rows
+    t0 = time.perf_counter()
+    oracle.rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, rows, nthreads=cores)
+    oracle.bwd_rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, g, rows, teacher=w.teacher_grads,
+                    nthreads=cores)
+    dt = time.perf_counter() - t0
+    if w.causal:
+        pairs = float(np.minimum(w.N_K, rows + (w.N_K - w.N_Q) + 1).sum())
+    else:
+        pairs = float(len(rows) * w.N_K)
+    per = step_flops(w) / (visible_pairs(w) * w.B * w.H)
+    return dt, per * pairs, len(rows)
+
+
+def rows_for(w, seconds: float, cores: int) -> int:
+    """Rows of one head the oracle processes in about `seconds` (two-point
+    calibration, so the fixed per-call cost does not inflate the estimate)."""
+    t1, _, n1 = oracle_sample(w, 32, 1, cores)
+    t2, _, n2 = oracle_sample(w, 256, 2, cores)
+    per_row = max((t2 - t1) / max(n2 - n1, 1), 1e-6)
+    fixed = max(t1 - per_row * n1, 0.0)
+    return int(min(w.N_Q, max(16, (seconds - fixed) / per_row)))
+
+
+def cpu_baseline(w, target_s: float = 15.0):
+    cores = cpu_cores()
+    dt, fl, n = oracle_sample(w, rows_for(w, target_s, cores), 3, cores)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} seeded query rows of head (0,0): forward plus full backward "
+                      f"({'teacher and student' if w.teacher_grads else 'student'} gradients) in fp64, "
+                      f"{dt:.1f} s wall, metric FLOPs counted over the rows' visible keys"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cores = cpu_cores()
+    total = args.steps + args.warmup
+    budget = 150.0                                  # seconds for the whole run
+    n_rows = rows_for(w, budget / total, cores)
+    for k in range(args.warmup):
+        oracle_sample(w, n_rows, 200 + k, cores)
+    tsum = fsum = 0.0
+    for k in range(args.steps):
+        dt, fl, n = oracle_sample(w, n_rows, 1000 + k, cores)
+        tsum += dt
+        fsum += fl
+    value = fsum / tsum / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tsum / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_rows} seeded query rows of head (0,0), forward plus full "
+                                   f"backward in fp64 on {cores} host threads"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w) -> dict:
+    in_bytes = 2 * w.B * w.H * (w.N_Q * (w.d_t + w.d_s) + w.N_K * (w.d_t + w.d_s))
+    return {"workload": w.name, "B": w.B, "H": w.H, "N_Q": w.N_Q, "N_K": w.N_K, "d_t": w.d_t, "d_s": w.d_s,
+            "causal": w.causal, "teacher_grads": w.teacher_grads, "student": w.student,
+            "flops_per_step": step_flops(w),
+            "l2": (f"inputs {in_bytes / 1e6:.0f} MB per step vs 126 MB L2; no flush"
+                   if in_bytes > L2_BYTES else "L2 flushed between steps (256 MB write)")}
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--workload", default="causal_8k_d128")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from attention_kl_divergence_attn_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import attention_kl_divergence_attn_b200 as skl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    # each rank solves its own independent problem (its own seed)
+    wr = dataclasses.replace(w, seed=w.seed + 7919 * rank)
+    host = [t.pin_memory() for t in inputs.make_inputs(wr)]
+    x = [t.to(dev, non_blocking=True) for t in host]
+    B, H, NQ, NK, dt_, ds_ = w.B, w.H, w.N_Q, w.N_K, w.d_t, w.d_s
+    f32 = dict(dtype=torch.float32, device=dev)
+    kl, lt, ls = (torch.empty(B, H, NQ, **f32) for _ in range(3))
+    loss = torch.empty((), **f32)
+    dqs, dks = torch.empty(B, H, NQ, ds_, **f32), torch.empty(B, H, NK, ds_, **f32)
+    dqt = torch.empty(B, H, NQ, dt_, **f32) if w.teacher_grads else None
+    dkt = torch.empty(B, H, NK, dt_, **f32) if w.teacher_grads else None
+    flush = None
+    if 2 * B * H * (NQ + NK) * (dt_ + ds_) <= L2_BYTES:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(stream=stream)
+
+    names = ["streamkl_fwd_kernel", "streamkl_mean_kernel", "streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"]
+
+    def step(ev=None):
+        if flush is not None:
+            flush.zero_()
+        if ev is not None:
+            ev[0].record(stream)
+        skl.streamkl_fwd(*x, w.scale_t, w.scale_s, w.causal, loss_mean=False, out=(kl, lt, ls), **kw)
+        if ev is not None:
+            ev[1].record(stream)
+        skl.streamkl_loss_mean(kl, out=loss, **kw)
+        if ev is not None:
+            ev[2].record(stream)
+        skl.streamkl_bwd_dk(*x, kl, lt, ls, w.scale_t, w.scale_s, w.causal, teacher_grads=w.teacher_grads,
+                            out=(dks, dkt), **kw)
+        if ev is not None:
+            ev[3].record(stream)
+        skl.streamkl_bwd_dq(*x, kl, lt, ls, w.scale_t, w.scale_s, w.causal, teacher_grads=w.teacher_grads,
+                            out=(dqs, dqt), **kw)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    skl.streamkl_check(stream)
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for k in range(K):
+            step(evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    per_kernel = {n: 0.0 for n in names}
+    for e in evs:
+        for i, n in enumerate(names):
+            per_kernel[n] += e[i].elapsed_time(e[i + 1])
+    per_kernel = {n: v / K for n, v in per_kernel.items()}
+    code = skl.streamkl_check(stream)
+
+    # end to end through the public API: pinned host inputs -> device, step, loss -> host
+    loss_h = torch.empty((), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host)
+
+    def e2e_step():
+        for dst, src in zip(x, host):
+            dst.copy_(src, non_blocking=True)
+        step()
+        loss_h.copy_(loss, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = e0.elapsed_time(e1)
+
+    if world > 1:
+        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total, ms_e2e = tt.tolist()
+
+    ms_step = ms_total / K
+    flops = step_flops(w)
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    e2e_value = flops * world / (ms_e2e / K * 1e-3) / 1e12
+
+    sustained, burst, peak_src = measured_peak()
+    kf = kernel_flops(w)
+    dominant = max((n for n in names if kf[n] > 0), key=lambda n: per_kernel[n])
+    achieved = kf[dominant] / (per_kernel[dominant] * 1e-3) / 1e12
+    traffic = recorded_traffic(dominant, w.name)
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            try:
+                cpu = cpu_baseline(w)
+            except Exception as exc:                 # the CPU leg must not hide the GPU number
+                cpu = {"value": None, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                       "sample": f"failed: {exc}"}
+        total_k = sum(per_kernel.values())
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w), parallelism=f"independent problem per GPU x{world}"),
+            "pct_of_nominal_bf16_peak": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
+            "pct_of_measured_bf16_peak": 100.0 * value / world / burst,
+            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": sustained,
+                         "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
+                         "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                         "flops_per_launch": kf[dominant]},
+            "kernels": {n: {"ms": per_kernel[n], "share": per_kernel[n] / total_k,
+                            "mma_tflops": (kf[n] / (per_kernel[n] * 1e-3) / 1e12) if kf[n] else None}
+                        for n in names},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
+            "gpu_launches": 4 * K,
+            "clocks": sampler.summary(),
+            "device_status": code,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

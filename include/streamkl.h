@@ -102,6 +102,31 @@ streamkl_status streamkl_bwd(const void *q_t, const void *k_t, const void *q_s, 
                              float *dq_s, float *dk_s, float *dq_t, float *dk_t,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * The two halves of streamkl_bwd, for callers that need only one side (a
+ * frozen query or key projection) or that schedule them separately.  Same
+ * arguments and meaning as streamkl_bwd.  streamkl_bwd_dk writes dk_s (and
+ * dk_t if non-NULL); streamkl_bwd_dq writes dq_s (and dq_t if non-NULL).
+ * Each recomputes both distributions on its own.
+ */
+streamkl_status streamkl_bwd_dk(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                                float scale_t, float scale_s, int causal,
+                                const float *kl, const float *lse_t, const float *lse_s,
+                                const float *dkl, float dloss, float *dk_s, float *dk_t,
+                                void *workspace, size_t workspace_bytes, void *stream);
+streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                                float scale_t, float scale_s, int causal,
+                                const float *kl, const float *lse_t, const float *lse_s,
+                                const float *dkl, float dloss, float *dq_s, float *dq_t,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* loss_mean (device scalar) = mean of kl[0..n_rows) in a fixed summation
+ * order (so repeated calls give identical bits); the same reduction
+ * streamkl_fwd runs when its loss_mean argument is non-NULL. */
+streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream);
+
 /* Clears the workspace (enqueued on `stream`).  Needed once per workspace. */
 streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 

@@ -51,6 +51,9 @@ def lib():
             L.streamkl_oracle_rows.argtypes = ([_D] * 4 + shape + [_I64, ctypes.c_int64, _D]
                                                + [_D] * 5 + [ctypes.c_int])
             L.streamkl_oracle_rows.restype = ctypes.c_int
+            L.streamkl_oracle_bwd_rows.argtypes = ([_D] * 4 + shape + [_D, _I64, ctypes.c_int64]
+                                                   + [_D] * 4 + [ctypes.c_int])
+            L.streamkl_oracle_bwd_rows.restype = ctypes.c_int
             L.streamkl_oracle_mean.argtypes = [_D, ctypes.c_int64]
             L.streamkl_oracle_mean.restype = ctypes.c_double
             _lib = L
@@ -136,6 +139,24 @@ def rows(qt, kt, qs, ks, scale_t, scale_s, causal, row_ids, g=None, teacher=Fals
         if teacher:
             out["dq_t"] = dqt.reshape(B * H * N_Q, d_t)[r]
     return out
+
+
+def bwd_rows(qt, kt, qs, ks, scale_t, scale_s, causal, g, row_ids, teacher=True, nthreads=0):
+    """Backward over the listed flat rows only: their dQ rows and their dK contributions."""
+    qt, kt, qs, ks = map(_f64, (qt, kt, qs, ks))
+    B, H, N_Q, N_K, d_t, d_s = _shape(qt, kt, qs, ks)
+    g = np.ascontiguousarray(np.broadcast_to(np.asarray(g, dtype=np.float64), (B, H, N_Q)))
+    r = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
+    dqs = np.zeros_like(qs); dks = np.zeros_like(ks)
+    dqt = np.zeros_like(qt) if teacher else None
+    dkt = np.zeros_like(kt) if teacher else None
+    rc = lib().streamkl_oracle_bwd_rows(_p(qt), _p(kt), _p(qs), _p(ks), B, H, N_Q, N_K, d_t, d_s,
+                                        float(scale_t), float(scale_s), int(bool(causal)), _p(g),
+                                        r.ctypes.data_as(_I64), int(r.size),
+                                        _p(dqs), _p(dks), _p(dqt), _p(dkt), int(nthreads))
+    if rc:
+        raise ValueError(f"oracle bwd_rows rejected the arguments (rc={rc})")
+    return dqs, dks, dqt, dkt
 
 
 def mean(kl) -> float:

@@ -252,6 +252,28 @@ int streamkl_oracle_rows(const double *q_t, const double *k_t, const double *q_s
     return run(w, n_rows, nthreads, NULL, NULL);
 }
 
+/* Backward restricted to the listed rows: their dQ rows and their
+ * contributions to dK (the dK of the rows not listed is left out).  Used to
+ * time the oracle on a bounded sample of a large problem. */
+int streamkl_oracle_bwd_rows(const double *q_t, const double *k_t, const double *q_s, const double *k_s,
+                             int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                             double scale_t, double scale_s, int causal, const double *g,
+                             const int64_t *rows, int64_t n_rows,
+                             double *dq_s, double *dk_s, double *dq_t, double *dk_t, int nthreads)
+{
+    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal) || !g) return 1;
+    for (int64_t k = 0; k < n_rows; ++k)
+        if (rows[k] < 0 || rows[k] >= (int64_t)B * H * N_Q) return 1;
+    work_t w;
+    memset(&w, 0, sizeof w);
+    w.q_t = q_t; w.k_t = k_t; w.q_s = q_s; w.k_s = k_s;
+    w.B = B; w.H = H; w.N_Q = N_Q; w.N_K = N_K; w.d_t = d_t; w.d_s = d_s; w.causal = causal;
+    w.scale_t = scale_t; w.scale_s = scale_s;
+    w.g = g; w.dq_s = dq_s; w.dq_t = dq_t;
+    w.rows = rows;
+    return run(w, n_rows, nthreads, dk_s, dk_t);
+}
+
 /* Mean of the per-row KL over every (b, h, i) row. */
 double streamkl_oracle_mean(const double *kl, int64_t n)
 {

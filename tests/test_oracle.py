@@ -288,3 +288,14 @@ def test_golden_tiny_regression():
     dqs, dks, _, _ = oracle.bwd(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, g=ref["g"], teacher=False)
     np.testing.assert_allclose(dqs.reshape(-1, 64)[0], ref["dq_s_row0"], rtol=1e-10, atol=1e-18)
     assert abs(np.linalg.norm(dks) - ref["norms"]["dk_s"]) < 1e-10 * ref["norms"]["dk_s"]
+
+
+def test_bwd_rows_partition_sums_to_full():
+    # the backward over two disjoint row sets adds up to the full backward
+    qt, kt, qs, ks = problem(N_Q=20, N_K=25, seed=47)
+    g = rand((1, 2, 20), 48)
+    full = oracle.bwd(qt, kt, qs, ks, 0.4, 0.3, True, g=g)
+    a = oracle.bwd_rows(qt, kt, qs, ks, 0.4, 0.3, True, g, np.arange(0, 40, 2))
+    b = oracle.bwd_rows(qt, kt, qs, ks, 0.4, 0.3, True, g, np.arange(1, 40, 2))
+    for f, x, y in zip(full, a, b):
+        np.testing.assert_allclose(x + y, f, rtol=1e-12, atol=1e-15)
