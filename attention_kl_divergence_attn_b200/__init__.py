@@ -60,6 +60,8 @@ def lib():
             L.streamkl_bwd_dq.restype = _I
             L.streamkl_loss_mean.argtypes = [_VP, ctypes.c_longlong, _VP, _VP]
             L.streamkl_loss_mean.restype = _I
+            L.streamkl_fwd_noalloc.argtypes = ([_VP] * 4 + shape + [_VP] * 4 + [_VP, ctypes.POINTER(ctypes.c_uint)])
+            L.streamkl_fwd_noalloc.restype = _I
             L.streamkl_workspace_size.argtypes = [_I] * 7
             L.streamkl_workspace_size.restype = ctypes.c_size_t
             L.streamkl_workspace_init.argtypes = [_VP, ctypes.c_size_t, _VP]

@@ -308,4 +308,65 @@ streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *los
     return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
+
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward without any caller-provided device memory.
+//
+// Some callers cannot allocate device memory at all, not even the small
+// workspace streamkl_fwd asks for: plug-in hosts that hand a library only the
+// buffers they planned in advance, runtimes that forbid allocation once they
+// are serving, and programs whose memory pool owns every byte of the device.
+// For them the workspace (the device status word) lives in this file-scope
+// array instead.  Every GPU that loads the library holds it until exit.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;   // fixed maximum scratch of this entry point
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};         // device address of the array, per device
+
+// Resolves the device address of the static array for the current device
+// (host code cannot use the symbol's name as a device pointer).
+streamkl_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return STREAMKL_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return STREAMKL_ERR_CUDA;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return STREAMKL_OK;
+}
+
+}  // namespace
+
+extern "C" streamkl_status streamkl_fwd_noalloc(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                                int B, int H, int N_Q, int N_K, int d_t, int d_s, float scale_t,
+                                                float scale_s, int causal, float *kl, float *lse_t, float *lse_s,
+                                                float *loss_mean, void *stream, unsigned int *status_out) {
+    if (streamkl_workspace_size(B, H, N_Q, N_K, d_t, d_s, causal) > kNoAllocScratchBytes)
+        return STREAMKL_ERR_WORKSPACE;          // this problem needs more scratch than the array holds
+    void *scratch = nullptr;
+    streamkl_status st = noalloc_scratch(&scratch);
+    if (st != STREAMKL_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the status word must start at zero for this call
+    if (cudaMemsetAsync(scratch, 0, kNoAllocScratchBytes, s) != cudaSuccess) return STREAMKL_ERR_CUDA;
+    st = streamkl_fwd(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s,
+                      loss_mean, scratch, kNoAllocScratchBytes, stream);
+    if (st != STREAMKL_OK || !status_out) return st;
+    // the caller asked for the device status: wait for this call and read it
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, scratch, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return STREAMKL_ERR_CUDA;
+    *status_out = word;
+    return (word & kStatusTimeout) ? STREAMKL_ERR_TIMEOUT : STREAMKL_OK;
+}

@@ -136,6 +136,37 @@ streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes,
  * pointer, nullable) receives the raw device status word (0 = clean). */
 streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int *code_out);
 
+/*
+ * Forward with no device memory from the caller beyond inputs and outputs.
+ * (An addition of this library; the paper has no counterpart.)
+ *
+ * For callers that cannot allocate device memory at all, not even the small
+ * workspace of streamkl_fwd: plug-in hosts that hand a library only buffers
+ * they planned in advance, runtimes that forbid allocation once serving, and
+ * programs whose memory pool owns the whole device.  Same arguments, results
+ * and errors as streamkl_fwd, but the status word lives in a fixed 256-byte
+ * array inside the library (a file-scope __device__ array that every GPU
+ * loading the library keeps until the process exits).  Nothing is allocated:
+ * no cudaMalloc, no cudaFree, no allocating library call.
+ *  - The first call on each device looks up that array's device address
+ *    (cudaGetSymbolAddress, with the device current); make that first call
+ *    before any stream capture.
+ *  - Each call clears the status word at its start.  All calls on a device
+ *    share the one array and it keeps the last call's contents, so calls that
+ *    overlap on the GPU (different streams, no ordering) race on it.
+ *  - A problem whose scratch need (streamkl_workspace_size) exceeds the array
+ *    is rejected with STREAMKL_ERR_WORKSPACE before anything is launched.
+ *  - status_out (host pointer): if non-NULL the call synchronises `stream`,
+ *    stores the device status word there (0 = clean) and returns
+ *    STREAMKL_ERR_TIMEOUT if a bounded wait gave up; if NULL the call returns
+ *    as soon as the work is enqueued.
+ */
+streamkl_status streamkl_fwd_noalloc(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                     int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                                     float scale_t, float scale_s, int causal,
+                                     float *kl, float *lse_t, float *lse_s, float *loss_mean,
+                                     void *stream, unsigned int *status_out);
+
 /* Static, human-readable name of a status. */
 const char *streamkl_strerror(streamkl_status status);
 
