@@ -19,10 +19,12 @@
 //       tiles: S^T = K Q^T for teacher and student (tcgen05, TMEM), dS^T in
 //       bf16 to shared memory, dK += dS^T Q accumulated in TMEM.  Thread =
 //       key row; per-query constants come from a small shared-memory table
-//       that the producer warp fills next to each TMA tile.
+//       that the producer warp fills next to each TMA tile.  Two gradient
+//       warpgroups split the 64 columns of a tile (32 each).
 //   streamkl_bwd_dq_kernel   CTA = 128 queries of one head; loops over 64-key
 //       tiles: S = Q K^T, dS in bf16 to shared memory, dQ += dS K in TMEM.
-//       Thread = query row; per-row constants live in registers.
+//       Thread = query row; per-row constants live in registers; two
+//       gradient warpgroups split the 64 columns of a tile.
 // Both recompute S: that costs one extra pair of QK^T products per element
 // but removes the fp32 read-modify-write traffic a single kernel would need
 // for the side it does not own.
@@ -73,6 +75,16 @@ __device__ __forceinline__ void store_row64(uint8_t *tile, int row, const uint32
     }
 }
 
+// Stores 32 bf16 (16 packed pairs) as 16-byte chunks chunk0..chunk0+3 of row `row`
+// of a [rows][64] 128B-swizzled tile.
+__device__ __forceinline__ void store_row32(uint8_t *tile, int row, int chunk0, const uint32_t (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((chunk0 + c) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    }
+}
+
 // Reads `ncols` fp32 accumulator columns of this thread's TMEM lane, scales them
 // and writes them to dst (one row, contiguous) if `store`.
 template <int NCOLS>
@@ -93,6 +105,8 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *ds
 }
 
 // ============================================================================ dK kernel
+constexpr int kBwdWarpgroups = 2;    // gradient warpgroups per CTA; each takes 32 columns of a tile
+
 template <int DT, int DS, bool TEACHER>
 struct DkvCfg {
     static constexpr int BN = 128, BM = 64;       // keys per CTA, queries per tile
@@ -109,7 +123,8 @@ struct DkvCfg {
     static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int NWG = kBwdWarpgroups;
+    static constexpr int THREADS = 64 + 128 * NWG;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_KS = idesc_bf16(128, DS, 0, 1);
     static constexpr uint32_t IDESC_KT = idesc_bf16(128, DT, 0, 1);
@@ -117,7 +132,7 @@ struct DkvCfg {
 };
 
 template <int DT, int DS, bool TEACHER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     streamkl_bwd_dkv_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
                             const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
                             const BwdParams p) {
@@ -152,9 +167,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4);
+            mbar_init(&bar_sempty[b], 4 * C::NWG);
         }
-        mbar_init(&bar_dsfull, 4);
+        mbar_init(&bar_dsfull, 4 * C::NWG);
         mbar_init(&bar_dsempty, 1);
         mbar_init(&bar_done, 1);
         abort_flag = 0;
@@ -268,10 +283,14 @@ __global__ void __launch_bounds__(192, 1)
             mma_commit(&bar_done);
         }
     } else {
-        // ------------------------------------------------------------ gradient warpgroup (thread = key)
+        // ------------------------------------------------------------ gradient warpgroups (thread = key)
+        // Warpgroup wg handles query columns [32 wg, 32 wg + 32) of every tile and
+        // drains its share of the dK columns at the end.
+        const int wg = (warp - 2) >> 2;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int gk = k0 + row;
+        const int c0 = wg * 32;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         bool ok = true;
         for (int t = 0; t < n_qt; ++t) {
@@ -280,38 +299,36 @@ __global__ void __launch_bounds__(192, 1)
             if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 16) ||
                 !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
             tc_fence_after();
-            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::STAGE_TMA);
-            const bool masked = p.causal && (k0 + C::BN - 1 > q0 + off);
-            const int qmin = gk - off - q0;        // first visible query column (causal)
-            uint32_t ps[32], pt[32];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::STAGE_TMA) + c0;
+            const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c0 + off);
+            const int qmin = gk - off - (q0 + c0);   // first visible query column of this warpgroup (causal)
+            uint32_t ps[16], pt[16];
+            {
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 128 + c * 32, ut);
-                tmem_ld32(lane_base + buf * 128 + 64 + c * 32, us);
+                tmem_ld32(lane_base + buf * 128 + c0, ut);
+                tmem_ld32(lane_base + buf * 128 + 64 + c0, us);
                 tmem_ld_wait();
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const int q = c * 32 + k;
-                    const float4 c0 = cst[q], c1 = cst[q + 1];
-                    float at0 = fmaf(ut[k], p.ct, -c0.x), at1 = fmaf(ut[k + 1], p.ct, -c1.x);
-                    float as0 = fmaf(us[k], p.cs, -c0.y), as1 = fmaf(us[k + 1], p.cs, -c1.y);
+                    const float4 e0 = cst[k], e1 = cst[k + 1];
+                    float at0 = fmaf(ut[k], p.ct, -e0.x), at1 = fmaf(ut[k + 1], p.ct, -e1.x);
+                    float as0 = fmaf(us[k], p.cs, -e0.y), as1 = fmaf(us[k + 1], p.cs, -e1.y);
                     float P0 = ex2(at0), P1 = ex2(at1), Q0 = ex2(as0), Q1 = ex2(as1);
                     if (masked) {
-                        if (q < qmin) { P0 = 0.f; Q0 = 0.f; }
-                        if (q + 1 < qmin) { P1 = 0.f; Q1 = 0.f; }
+                        if (k < qmin) { P0 = 0.f; Q0 = 0.f; }
+                        if (k + 1 < qmin) { P1 = 0.f; Q1 = 0.f; }
                     }
-                    ps[q >> 1] = pack_bf16(c0.z * (Q0 - P0), c1.z * (Q1 - P1));
+                    ps[k >> 1] = pack_bf16(e0.z * (Q0 - P0), e1.z * (Q1 - P1));
                     if (TEACHER)
-                        pt[q >> 1] = pack_bf16((c0.z * P0) * ((at0 - as0) - c0.w), (c1.z * P1) * ((at1 - as1) - c1.w));
+                        pt[k >> 1] = pack_bf16((e0.z * P0) * ((at0 - as0) - e0.w), (e1.z * P1) * ((at1 - as1) - e1.w));
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_sempty[buf]);
             if (t > 0 && !mbar_wait(&bar_dsempty, (t - 1) & 1, p.st, abort_v, 18)) { ok = false; break; }
-            store_row64(sDss, row, ps);
-            if (TEACHER) store_row64(sDst, row, pt);
+            store_row32(sDss, row, wg * 4, ps);
+            if (TEACHER) store_row32(sDst, row, wg * 4, pt);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_dsfull);
@@ -320,9 +337,10 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const bool store = gk < p.N_K;
             const size_t r = (size_t)bh * p.N_K + (store ? gk : 0);
-            drain_row<DS>(lane_base + C::TMEM_DKS, p.out_s, p.dk_s + r * DS, store);
-            if (TEACHER) drain_row<DT>(lane_base + C::TMEM_DKT, p.out_t, p.dk_t + r * DT, store);
-        } else if (n_qt == 0 && gk < p.N_K) {
+            constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
+            drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s, p.dk_s + r * DS + wg * HS, store);
+            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t, p.dk_t + r * DT + wg * HT, store);
+        } else if (n_qt == 0 && gk < p.N_K && wg == 0) {
             const size_t r = (size_t)bh * p.N_K + gk;
             for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
             if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[r * DT + c] = 0.f;
@@ -352,7 +370,8 @@ struct DqCfg {
     static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int NWG = kBwdWarpgroups;
+    static constexpr int THREADS = 64 + 128 * NWG;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_QS = idesc_bf16(128, DS, 0, 1);
     static constexpr uint32_t IDESC_QT = idesc_bf16(128, DT, 0, 1);
@@ -360,7 +379,7 @@ struct DqCfg {
 };
 
 template <int DT, int DS, bool TEACHER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     streamkl_bwd_dq_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
                            const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
                            const BwdParams p) {
@@ -395,9 +414,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4);
+            mbar_init(&bar_sempty[b], 4 * C::NWG);
         }
-        mbar_init(&bar_dsfull, 4);
+        mbar_init(&bar_dsfull, 4 * C::NWG);
         mbar_init(&bar_dsempty, 1);
         mbar_init(&bar_done, 1);
         abort_flag = 0;
@@ -492,10 +511,14 @@ __global__ void __launch_bounds__(192, 1)
             mma_commit(&bar_done);
         }
     } else {
-        // ------------------------------------------------------------ gradient warpgroup (thread = query)
+        // ------------------------------------------------------------ gradient warpgroups (thread = query)
+        // Warpgroup wg handles key columns [32 wg, 32 wg + 32) of every tile and
+        // drains its share of the dQ columns at the end.
+        const int wg = (warp - 2) >> 2;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int gq = q0 + row;
+        const int c0 = wg * 32;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         float Lt = 0.f, Ls = 0.f, g = 0.f, KL2 = 0.f;
         if (gq < p.N_Q) {
@@ -511,35 +534,34 @@ __global__ void __launch_bounds__(192, 1)
             const int buf = kt & 1, use = kt >> 1;
             if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 26)) { ok = false; break; }
             tc_fence_after();
-            const int kb = kt * C::BN;
-            const bool masked = (kb + C::BN > p.N_K) || (p.causal && (kb + C::BN - 1 > q0 + off));
-            uint32_t ps[32], pt[32];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            const int kb = kt * C::BN + c0;
+            const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
+            uint32_t ps[16], pt[16];
+            {
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 128 + c * 32, ut);
-                tmem_ld32(lane_base + buf * 128 + 64 + c * 32, us);
+                tmem_ld32(lane_base + buf * 128 + c0, ut);
+                tmem_ld32(lane_base + buf * 128 + 64 + c0, us);
                 tmem_ld_wait();
                 if (masked) {
 #pragma unroll
                     for (int k = 0; k < 32; k += 2) {
-                        const int j = kb + c * 32 + k;
+                        const int j = kb + k;
                         ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Ls, g, KL2, j < lim,
-                                               j + 1 < lim, ps[(c * 32 + k) >> 1], pt[(c * 32 + k) >> 1]);
+                                               j + 1 < lim, ps[k >> 1], pt[k >> 1]);
                     }
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; k += 2)
                         ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Ls, g, KL2, true,
-                                                true, ps[(c * 32 + k) >> 1], pt[(c * 32 + k) >> 1]);
+                                                true, ps[k >> 1], pt[k >> 1]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_sempty[buf]);
             if (kt > 0 && !mbar_wait(&bar_dsempty, (kt - 1) & 1, p.st, abort_v, 27)) { ok = false; break; }
-            store_row64(sDss, row, ps);
-            if (TEACHER) store_row64(sDst, row, pt);
+            store_row32(sDss, row, wg * 4, ps);
+            if (TEACHER) store_row32(sDst, row, wg * 4, pt);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_dsfull);
@@ -548,8 +570,9 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const bool store = gq < p.N_Q;
             const size_t r = (size_t)bh * p.N_Q + (store ? gq : 0);
-            drain_row<DS>(lane_base + C::TMEM_DQS, p.out_s, p.dq_s + r * DS, store);
-            if (TEACHER) drain_row<DT>(lane_base + C::TMEM_DQT, p.out_t, p.dq_t + r * DT, store);
+            constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
+            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s, p.dq_s + r * DS + wg * HS, store);
+            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t, p.dq_t + r * DT + wg * HT, store);
         }
     }
 

@@ -5,17 +5,19 @@
 // query-key tiles through on-chip memory with an online formulation of the
 // coupled two-distribution KL reduction, so neither softmax is materialised.
 //
-// One CTA owns 128 query rows of one (batch, head).  Roles (6 warps):
+// One CTA owns 128 query rows of one (batch, head).  Roles (2 + 4*NWG warps):
 //   warp 0      TMA producer: Q_t, Q_s once; K_t, K_s tiles of 128 keys into
 //               an NSTAGE-deep shared-memory ring.
 //   warp 1      MMA issuer (one elected thread) and TMEM owner: per key tile
 //               S_t = Q_t K_t^T and S_s = Q_s K_s^T as tcgen05.mma (bf16 in,
 //               fp32 accumulate) into one of two TMEM buffers (2 x 256 cols).
-//   warps 2..5  softmax warpgroup: thread = query row = TMEM lane.  It reads
-//               its row of both logit tiles in 32-column chunks (tcgen05.ld
-//               32x32b), and updates the per-row online state
-//               (M_t, l_t, A, M_s, l_s); row reductions are thread-local
-//               because the 32x32b layout gives each thread one whole row.
+//   warps 2..   NWG softmax warpgroups: thread = query row = TMEM lane.  Each
+//               warpgroup reads its 128/NWG key columns of both logit tiles
+//               in 32-column chunks (tcgen05.ld 32x32b) and updates its own
+//               per-row online state (M_t, l_t, A, M_s, l_s); row reductions
+//               are thread-local because the 32x32b layout gives each thread
+//               one whole row.  The warpgroups' states are merged at the end
+//               (the state is associative: rescale both to the larger max).
 // State (log2 units, y = scale * log2(e) * q.k):
 //   M_t, M_s  running maxima of y_t, y_s
 //   l_t = sum 2^(y_t - M_t),  l_s = sum 2^(y_s - M_s)
@@ -35,7 +37,7 @@ struct FwdParams {
     DevStatus st;
 };
 
-template <int DT, int DS>
+template <int DT, int DS, int NWG>
 struct FwdCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int BLK = 128 * 128;                    // one [128 rows][64] bf16 box
@@ -46,9 +48,11 @@ struct FwdCfg {
     static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
     static constexpr int SMEM = Q_BYTES + NSTAGE * STAGE_BYTES + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 64 + 128 * NWG;           // TMA warp, MMA warp, NWG softmax warpgroups
+    static constexpr int CW = BN / NWG;                      // key columns of a tile per warpgroup
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+    static_assert(CW % 32 == 0, "each warpgroup reads whole 32-column chunks");
 };
 
 // Number of key tiles a 128-row query tile starting at q0 must visit.
@@ -100,12 +104,12 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
     Ms = Ms_new;
 }
 
-template <int DT, int DS>
-__global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
+template <int DT, int DS, int NWG>
+__global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     streamkl_fwd_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
                         const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
                         const FwdParams p) {
-    using C = FwdCfg<DT, DS>;
+    using C = FwdCfg<DT, DS, NWG>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQt = smem;
@@ -115,6 +119,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
     __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_sempty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
+    __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // heaviest (latest) causal query tiles first
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4);
+            mbar_init(&bar_sempty[b], 4 * NWG);
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -210,23 +215,28 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax warpgroup
+        // ------------------------------------------------------------ softmax warpgroups
+        // Warpgroup wg reads key columns [wg*CW, (wg+1)*CW) of every tile for all 128 rows
+        // (warp w may only touch TMEM lanes 32*(w%4)..+31); the per-row states of the
+        // warpgroups are merged at the end with the associative rule of the recurrence.
+        const int wg = (warp - 2) >> 2;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int grow = q0 + row;
+        const int c0 = wg * C::CW;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
         for (int kt = 0; kt < n_kt; ++kt) {
             const int buf = kt & 1, use = kt >> 1;
             if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 5)) break;
             tc_fence_after();
-            const int k0 = kt * C::BN;
-            const bool masked = (k0 + C::BN > p.N_K) || (p.causal && (k0 + C::BN - 1 > q0 + off));
+            const int k0 = kt * C::BN + c0;
+            const bool masked = (k0 + C::CW > p.N_K) || (p.causal && (k0 + C::CW - 1 > q0 + off));
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < C::CW / 32; ++c) {
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 256 + c * 32, ut);
-                tmem_ld32(lane_base + buf * 256 + 128 + c * 32, us);
+                tmem_ld32(lane_base + buf * 256 + c0 + c * 32, ut);
+                tmem_ld32(lane_base + buf * 256 + 128 + c0 + c * 32, us);
                 tmem_ld_wait();
                 if (masked) {
                     const int lim = p.causal ? min(p.N_K, grow + off + 1) : p.N_K;   // first hidden key
@@ -243,7 +253,30 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_sempty[buf]);
         }
-        if (grow < p.N_Q && !*abort_v) {
+        if (NWG > 1) {
+            if (wg > 0) {
+                merge[wg - 1][0][row] = Mt; merge[wg - 1][1][row] = Ms; merge[wg - 1][2][row] = lt;
+                merge[wg - 1][3][row] = ls; merge[wg - 1][4][row] = A;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(128 * NWG) : "memory");
+            if (wg == 0) {
+#pragma unroll
+                for (int o = 0; o < NWG - 1; ++o) {
+                    const float Mt2 = merge[o][0][row], Ms2 = merge[o][1][row];
+                    const float nMt = fmaxf(Mt, Mt2), nMs = fmaxf(Ms, Ms2);
+                    if (nMt != -INFINITY) {
+                        const float a1 = ex2(Mt - nMt), a2 = ex2(Mt2 - nMt);
+                        const float b1 = ex2(Ms - nMs), b2 = ex2(Ms2 - nMs);
+                        lt = lt * a1 + merge[o][2][row] * a2;
+                        A = A * a1 + merge[o][4][row] * a2;
+                        ls = ls * b1 + merge[o][3][row] * b2;
+                        Mt = nMt;
+                        Ms = nMs;
+                    }
+                }
+            }
+        }
+        if (wg == 0 && grow < p.N_Q && !*abort_v) {
             const float LN2 = 0.69314718055994530942f;
             const float lse_t2 = Mt + lg2(lt), lse_s2 = Ms + lg2(ls);
             const size_t r = (size_t)bh * p.N_Q + grow;

@@ -82,11 +82,13 @@ cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+constexpr int kFwdWarpgroups = 2;
+
 template <int DT, int DS>
 streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const CUtensorMap &qs,
                            const CUtensorMap &ks, const FwdParams &p, cudaStream_t stream) {
-    using C = FwdCfg<DT, DS>;
-    auto kern = streamkl_fwd_kernel<DT, DS>;
+    using C = FwdCfg<DT, DS, kFwdWarpgroups>;
+    auto kern = streamkl_fwd_kernel<DT, DS, kFwdWarpgroups>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
     const long long grid = (long long)p.BH * p.n_qt;
     kern<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
