@@ -16,18 +16,27 @@
 // accumulates in tensor memory and is written exactly once (no atomics, and a
 // deterministic result):
 //   streamkl_bwd_dkv_kernel  CTA = 128 keys of one head; loops over 64-query
-//       tiles: S^T = K Q^T for teacher and student (tcgen05, TMEM), dS^T in
-//       bf16 to shared memory, dK += dS^T Q accumulated in TMEM.  Thread =
-//       key row; per-query constants come from a small shared-memory table
-//       that the producer warp fills next to each TMA tile.  Two gradient
-//       warpgroups split the 64 columns of a tile (32 each).
+//       tiles: S^T = K Q^T (teacher and student), dS^T, dK += dS^T Q.
+//       Thread = key row; per-query constants come from a small shared-memory
+//       table the producer warp fills next to each TMA tile of Q.
 //   streamkl_bwd_dq_kernel   CTA = 128 queries of one head; loops over 64-key
-//       tiles: S = Q K^T, dS in bf16 to shared memory, dQ += dS K in TMEM.
-//       Thread = query row; per-row constants live in registers; two
-//       gradient warpgroups split the 64 columns of a tile.
+//       tiles: S = Q K^T, dS, dQ += dS K.  Thread = query row; per-row
+//       constants live in registers.
 // Both recompute S: that costs one extra pair of QK^T products per element
 // but removes the fp32 read-modify-write traffic a single kernel would need
-// for the side it does not own.
+// for the side it does not own (measured at ~5.8 TB/s of L2 reductions on
+// B200, that traffic would cost more than the recompute).
+//
+// Pipeline (both kernels).  Gradient warpgroups ping-pong over tiles: tile t
+// goes to TMEM buffer t & 1 (S_t in columns [0,64), S_s in [64,128) of the
+// buffer) and to the warpgroups of parity t & 1; with NH = 2 halves per parity
+// each of those warpgroups takes 32 of the tile's 64 columns.  A warpgroup
+// reads its S columns in 32-column chunks and writes the chunk's bf16 dS
+// (16 packed columns) over the first half of the same chunk, which only it
+// reads; the MMA warp then uses those columns directly as the A operand of
+// the gradient MMA (tcgen05.mma with A in tensor memory), so dS never touches
+// shared memory.  Because MMAs issued by one thread execute in order, S of
+// tile t+2 can be issued into buffer t & 1 right after the gradient MMA of t.
 #pragma once
 
 #include "sm100.cuh"
@@ -46,67 +55,52 @@ struct BwdParams {
 
 constexpr float kLog2eF = 1.4426950408889634074f;
 
-// dS for two adjacent elements, packed as bf16x2.
+// dS for two adjacent elements, packed as bf16x2 (lower half = first element).
+// Per-element constants: L (log2-domain LSEs), g and KL*log2(e).
 template <bool TEACHER, bool MASKED>
-__device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float us1, float ct, float cs, float Lt,
-                                        float Ls, float g, float KL2, bool vis0, bool vis1, uint32_t &ps,
-                                        uint32_t &pt) {
-    const float at0 = fmaf(ut0, ct, -Lt), at1 = fmaf(ut1, ct, -Lt);
-    const float as0 = fmaf(us0, cs, -Ls), as1 = fmaf(us1, cs, -Ls);
+__device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float us1, float ct, float cs, float Lt0,
+                                        float Lt1, float Ls0, float Ls1, float g0, float g1, float K0, float K1,
+                                        bool vis0, bool vis1, uint32_t &ps, uint32_t &pt) {
+    const float at0 = fmaf(ut0, ct, -Lt0), at1 = fmaf(ut1, ct, -Lt1);
+    const float as0 = fmaf(us0, cs, -Ls0), as1 = fmaf(us1, cs, -Ls1);
     float P0 = ex2(at0), P1 = ex2(at1);
     float Q0 = ex2(as0), Q1 = ex2(as1);
     if (MASKED) {
         P0 = vis0 ? P0 : 0.f; Q0 = vis0 ? Q0 : 0.f;
         P1 = vis1 ? P1 : 0.f; Q1 = vis1 ? Q1 : 0.f;
     }
-    ps = pack_bf16(g * (Q0 - P0), g * (Q1 - P1));
-    if (TEACHER) {
-        const float gP0 = g * P0, gP1 = g * P1;
-        pt = pack_bf16(gP0 * ((at0 - as0) - KL2), gP1 * ((at1 - as1) - KL2));
-    }
+    ps = pack_bf16(g0 * (Q0 - P0), g1 * (Q1 - P1));
+    if (TEACHER) pt = pack_bf16((g0 * P0) * ((at0 - as0) - K0), (g1 * P1) * ((at1 - as1) - K1));
 }
 
-// Stores 64 bf16 (32 packed pairs) as row `row` of a [rows][64] 128B-swizzled tile.
-__device__ __forceinline__ void store_row64(uint8_t *tile, int row, const uint32_t (&v)[32]) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint32_t off = (uint32_t)row * 128u + ((uint32_t)(c ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-    }
-}
-
-// Stores 32 bf16 (16 packed pairs) as 16-byte chunks chunk0..chunk0+3 of row `row`
-// of a [rows][64] 128B-swizzled tile.
-__device__ __forceinline__ void store_row32(uint8_t *tile, int row, int chunk0, const uint32_t (&v)[16]) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((chunk0 + c) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-    }
-}
-
-// Reads `ncols` fp32 accumulator columns of this thread's TMEM lane, scales them
-// and writes them to dst (one row, contiguous) if `store`.
+// Reads `NCOLS` (a multiple of 16) fp32 accumulator columns of this thread's
+// TMEM lane, scales them and writes them to dst (one row, contiguous) if `store`.
 template <int NCOLS>
 __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool store) {
 #pragma unroll 1
-    for (int c = 0; c < NCOLS / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + c * 32, v);
+    for (int c = 0; c < NCOLS / 16; ++c) {
+        float v[16];
+        tmem_ld16(taddr + c * 16, v);
         tmem_ld_wait();
         if (store) {
-            float4 *d4 = reinterpret_cast<float4 *>(dst + c * 32);
+            float4 *d4 = reinterpret_cast<float4 *>(dst + c * 16);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < 4; ++k)
                 d4[k] = make_float4(v[4 * k] * scale, v[4 * k + 1] * scale, v[4 * k + 2] * scale,
                                     v[4 * k + 3] * scale);
         }
     }
 }
 
-// ============================================================================ dK kernel
-constexpr int kBwdWarpgroups = 2;    // gradient warpgroups per CTA; each takes 32 columns of a tile
+// TMEM column (within a 64-column half of a buffer) of the packed bf16 dS for
+// keys/queries [16 ks, 16 ks + 16): chunk ks/2 keeps its dS in the first 16 of
+// its 32 columns.
+__host__ __device__ constexpr uint32_t ds_col(int ks) { return (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8); }
 
+constexpr int kBwdParities = 2;      // ping-pong: tiles alternate between two TMEM buffers
+constexpr int kBwdHalves = 2;        // warpgroups per parity, each taking 64 / kBwdHalves columns
+
+// ============================================================================ dK kernel
 template <int DT, int DS, bool TEACHER>
 struct DkvCfg {
     static constexpr int BN = 128, BM = 64;       // keys per CTA, queries per tile
@@ -117,13 +111,11 @@ struct DkvCfg {
     static constexpr int CONST_BYTES = BM * 16;   // float4 per query
     static constexpr int STAGE_TMA = QT_BYTES + QS_BYTES;
     static constexpr int STAGE_BYTES = STAGE_TMA + CONST_BYTES;
-    static constexpr int DSB = BN * BM * 2;        // one dS^T tile, bf16
-    static constexpr int DS_BYTES = DSB * (TEACHER ? 2 : 1);
-    static constexpr int FIXED = KT_BYTES + KS_BYTES + DS_BYTES;
+    static constexpr int FIXED = KT_BYTES + KS_BYTES;
     static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
-    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
+    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
-    static constexpr int NWG = kBwdWarpgroups;
+    static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BM / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_KS = idesc_bf16(128, DS, 0, 1);
@@ -141,12 +133,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sKt = smem;
     uint8_t *sKs = sKt + C::KT_BYTES;
-    uint8_t *sDss = sKs + C::KS_BYTES;             // dS_s^T  [128 keys][64 queries]
-    uint8_t *sDst = sDss + C::DSB;                 // dS_t^T  (teacher)
-    uint8_t *sQ = sKs + C::KS_BYTES + C::DS_BYTES; // stages: Q_t, Q_s, constants
+    uint8_t *sQ = sKs + C::KS_BYTES;               // stages: Q_t, Q_s, per-query constants
 
-    __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_sempty[2];
-    __shared__ uint64_t bar_dsfull, bar_dsempty, bar_done;
+    __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
+    __shared__ uint64_t bar_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -167,10 +157,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4 * C::NWG);
+            mbar_init(&bar_dsfull[b], 4 * C::NH);
         }
-        mbar_init(&bar_dsfull, 4 * C::NWG);
-        mbar_init(&bar_dsempty, 1);
         mbar_init(&bar_done, 1);
         abort_flag = 0;
         fence_barrier_init();
@@ -215,7 +203,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             for (int h = 0; h < 2; ++h) {
                 const int q = lane + 32 * h;
                 const int i = q0 + q;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
                 if (i < p.N_Q) {
                     const size_t r = (size_t)bh * p.N_Q + i;
                     v.x = p.lse_t[r] * kLog2eF;
@@ -238,100 +226,98 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Descriptors are built once (warp-uniform) and advanced by constant offsets.
+        const uint64_t dKt = sw128_desc(smem_u32(sKt), 16, 1024), dKs = sw128_desc(smem_u32(sKs), 16, 1024);
+        const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);          // K-major view of a stage
+        const uint64_t dQ0mn = sw128_desc(smem_u32(sQ), C::QBLK, 1024);   // MN-major view of a stage
         if (elect_one()) {
-            const uint32_t aKt = smem_u32(sKt), aKs = smem_u32(sKs);
-            const uint32_t aDss = smem_u32(sDss), aDst = smem_u32(sDst);
+            // S^T of tile t into buffer t & 1
             auto issue_s = [&](int t) -> bool {
-                const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1, use = t >> 1;
+                const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
                 if (!mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 12)) return false;
-                if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, p.st, abort_v, 13)) return false;
                 tc_fence_after();
-                const uint32_t aQt = smem_u32(sQ + s * C::STAGE_BYTES), aQs = aQt + C::QT_BYTES;
+                const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES), dQs = desc_add(dQt, C::QT_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, sw128_desc(aKt + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024),
-                                sw128_desc(aQt + (kk >> 2) * C::QBLK + (kk & 3) * 32, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32),
+                                desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128 + 64,
-                                sw128_desc(aKs + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024),
-                                sw128_desc(aQs + (kk >> 2) * C::QBLK + (kk & 3) * 32, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32),
+                                desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
                 mma_commit(&bar_sfull[buf]);
                 return true;
             };
             bool ok = mbar_wait(&bar_k, 0, p.st, abort_v, 14);
             if (ok && n_qt > 0) ok = issue_s(0);
+            if (ok && n_qt > 1) ok = issue_s(1);
             for (int t = 0; ok && t < n_qt; ++t) {
-                if (t + 1 < n_qt && !issue_s(t + 1)) break;
-                if (!mbar_wait(&bar_dsfull, t & 1, p.st, abort_v, 15)) break;
+                const int buf = t & 1, s = t % C::NSTAGE;
+                if (!mbar_wait(&bar_dsfull[buf], (t >> 1) & 1, p.st, abort_v, 15)) break;
                 tc_fence_after();
-                const int s = t % C::NSTAGE;
-                const uint32_t aQt = smem_u32(sQ + s * C::STAGE_BYTES), aQs = aQt + C::QT_BYTES;
+                const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
+                // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BM / 16; ++ks)
-                    mma_bf16_ss(tmem + C::TMEM_DKS, sw128_desc(aDss + ks * 32, 16, 1024),
-                                sw128_desc(aQs + ks * 2048, C::QBLK, 1024), C::IDESC_KS, (t > 0 || ks > 0));
+                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
+                                (t > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BM / 16; ++ks)
-                        mma_bf16_ss(tmem + C::TMEM_DKT, sw128_desc(aDst + ks * 32, 16, 1024),
-                                    sw128_desc(aQt + ks * 2048, C::QBLK, 1024), C::IDESC_KT, (t > 0 || ks > 0));
+                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + 64 + ds_col(ks), desc_add(mQt, ks * 2048),
+                                    C::IDESC_KT, (t > 0 || ks > 0));
                 }
-                mma_commit(&bar_dsempty);
                 mma_commit(&bar_qempty[s]);
+                if (t + 2 < n_qt && !issue_s(t + 2)) break;
             }
             mma_commit(&bar_done);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = key)
-        // Warpgroup wg handles query columns [32 wg, 32 wg + 32) of every tile and
-        // drains its share of the dK columns at the end.
         const int wg = (warp - 2) >> 2;
+        const int par = wg % kBwdParities, half = wg / kBwdParities;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int gk = k0 + row;
-        const int c0 = wg * 32;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        const uint32_t bufc = lane_base + par * 128;  // this warpgroup's TMEM buffer
         bool ok = true;
-        for (int t = 0; t < n_qt; ++t) {
-            const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1, use = t >> 1;
+        for (int t = par; t < n_qt; t += kBwdParities) {
+            const int s = t % C::NSTAGE, n = t / C::NSTAGE;
             const int q0 = (first_qt + t) * C::BM;
-            if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 16) ||
+            if (!mbar_wait(&bar_sfull[par], (t >> 1) & 1, p.st, abort_v, 16) ||
                 !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
             tc_fence_after();
-            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::STAGE_TMA) + c0;
-            const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c0 + off);
-            const int qmin = gk - off - (q0 + c0);   // first visible query column of this warpgroup (causal)
-            uint32_t ps[16], pt[16];
-            {
+            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::STAGE_TMA);
+            const int qmin = gk - off - q0;        // first visible query column (causal)
+#pragma unroll
+            for (int cc = 0; cc < C::CW / 32; ++cc) {
+                const int c = half * (C::CW / 32) + cc;   // chunk of the tile
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 128 + c0, ut);
-                tmem_ld32(lane_base + buf * 128 + 64 + c0, us);
+                tmem_ld32(bufc + c * 32, ut);
+                tmem_ld32(bufc + 64 + c * 32, us);
                 tmem_ld_wait();
+                const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c * 32 + off);
+                uint32_t ps[16], pt[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const float4 e0 = cst[k], e1 = cst[k + 1];
-                    float at0 = fmaf(ut[k], p.ct, -e0.x), at1 = fmaf(ut[k + 1], p.ct, -e1.x);
-                    float as0 = fmaf(us[k], p.cs, -e0.y), as1 = fmaf(us[k + 1], p.cs, -e1.y);
-                    float P0 = ex2(at0), P1 = ex2(at1), Q0 = ex2(as0), Q1 = ex2(as1);
-                    if (masked) {
-                        if (k < qmin) { P0 = 0.f; Q0 = 0.f; }
-                        if (k + 1 < qmin) { P1 = 0.f; Q1 = 0.f; }
-                    }
-                    ps[k >> 1] = pack_bf16(e0.z * (Q0 - P0), e1.z * (Q1 - P1));
-                    if (TEACHER)
-                        pt[k >> 1] = pack_bf16((e0.z * P0) * ((at0 - as0) - e0.w), (e1.z * P1) * ((at1 - as1) - e1.w));
+                    const int q = c * 32 + k;
+                    const float4 e0 = cst[q], e1 = cst[q + 1];
+                    if (masked)
+                        ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y, e1.y,
+                                               e0.z, e1.z, e0.w, e1.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
+                    else
+                        ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
+                                                e1.y, e0.z, e1.z, e0.w, e1.w, true, true, ps[k >> 1], pt[k >> 1]);
                 }
+                // the columns written here were read by this chunk's (already completed) loads
+                tmem_st16(bufc + c * 32, ps);
+                if (TEACHER) tmem_st16(bufc + 64 + c * 32, pt);
             }
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sempty[buf]);
-            if (t > 0 && !mbar_wait(&bar_dsempty, (t - 1) & 1, p.st, abort_v, 18)) { ok = false; break; }
-            store_row32(sDss, row, wg * 4, ps);
-            if (TEACHER) store_row32(sDst, row, wg * 4, pt);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull);
+            if (lane == 0) mbar_arrive(&bar_dsfull[par]);
         }
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
@@ -364,13 +350,11 @@ struct DqCfg {
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
-    static constexpr int DSB = BM * BN * 2;
-    static constexpr int DS_BYTES = DSB * (TEACHER ? 2 : 1);
-    static constexpr int FIXED = QT_BYTES + QS_BYTES + DS_BYTES;
+    static constexpr int FIXED = QT_BYTES + QS_BYTES;
     static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
-    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
+    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
-    static constexpr int NWG = kBwdWarpgroups;
+    static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BN / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_QS = idesc_bf16(128, DS, 0, 1);
@@ -388,12 +372,10 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQt = smem;
     uint8_t *sQs = sQt + C::QT_BYTES;
-    uint8_t *sDss = sQs + C::QS_BYTES;             // dS_s [128 queries][64 keys]
-    uint8_t *sDst = sDss + C::DSB;
-    uint8_t *sK = sQs + C::QS_BYTES + C::DS_BYTES; // stages: K_t, K_s
+    uint8_t *sK = sQs + C::QS_BYTES;               // stages: K_t, K_s
 
-    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_sempty[2];
-    __shared__ uint64_t bar_dsfull, bar_dsempty, bar_done;
+    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
+    __shared__ uint64_t bar_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -414,10 +396,8 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4 * C::NWG);
+            mbar_init(&bar_dsfull[b], 4 * C::NH);
         }
-        mbar_init(&bar_dsfull, 4 * C::NWG);
-        mbar_init(&bar_dsempty, 1);
         mbar_init(&bar_done, 1);
         abort_flag = 0;
         fence_barrier_init();
@@ -466,60 +446,61 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Descriptors are built once (warp-uniform) and advanced by constant offsets.
+        const uint64_t dQt = sw128_desc(smem_u32(sQt), 16, 1024), dQs = sw128_desc(smem_u32(sQs), 16, 1024);
+        const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);          // K-major view of a stage
+        const uint64_t dK0mn = sw128_desc(smem_u32(sK), C::KBLK, 1024);   // MN-major view of a stage
         if (elect_one()) {
-            const uint32_t aQt = smem_u32(sQt), aQs = smem_u32(sQs);
-            const uint32_t aDss = smem_u32(sDss), aDst = smem_u32(sDst);
+            // S of key tile kt into buffer kt & 1
             auto issue_s = [&](int kt) -> bool {
-                const int s = kt % C::NSTAGE, n = kt / C::NSTAGE, buf = kt & 1, use = kt >> 1;
+                const int s = kt % C::NSTAGE, n = kt / C::NSTAGE, buf = kt & 1;
                 if (!mbar_wait(&bar_kfull[s], n & 1, p.st, abort_v, 22)) return false;
-                if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, p.st, abort_v, 23)) return false;
                 tc_fence_after();
-                const uint32_t aKt = smem_u32(sK + s * C::STAGE_BYTES), aKs = aKt + C::KT_BYTES;
+                const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES), dKs = desc_add(dKt, C::KT_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, sw128_desc(aQt + (kk >> 2) * C::QBLK + (kk & 3) * 32, 16, 1024),
-                                sw128_desc(aKt + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_bf16_ss(tmem + buf * 128, desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32),
+                                desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128 + 64,
-                                sw128_desc(aQs + (kk >> 2) * C::QBLK + (kk & 3) * 32, 16, 1024),
-                                sw128_desc(aKs + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32),
+                                desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
                 mma_commit(&bar_sfull[buf]);
                 return true;
             };
             bool ok = mbar_wait(&bar_q, 0, p.st, abort_v, 24);
             if (ok) ok = issue_s(0);
+            if (ok && n_kt > 1) ok = issue_s(1);
             for (int kt = 0; ok && kt < n_kt; ++kt) {
-                if (kt + 1 < n_kt && !issue_s(kt + 1)) break;
-                if (!mbar_wait(&bar_dsfull, kt & 1, p.st, abort_v, 25)) break;
+                const int buf = kt & 1, s = kt % C::NSTAGE;
+                if (!mbar_wait(&bar_dsfull[buf], (kt >> 1) & 1, p.st, abort_v, 25)) break;
                 tc_fence_after();
-                const int s = kt % C::NSTAGE;
-                const uint32_t aKt = smem_u32(sK + s * C::STAGE_BYTES), aKs = aKt + C::KT_BYTES;
+                const uint64_t mKt = desc_add(dK0mn, s * C::STAGE_BYTES), mKs = desc_add(mKt, C::KT_BYTES);
+                // dQ_s += dS_s K_s : A = dS_s from TMEM (buffer columns [0,32)), B = K_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks)
-                    mma_bf16_ss(tmem + C::TMEM_DQS, sw128_desc(aDss + ks * 32, 16, 1024),
-                                sw128_desc(aKs + ks * 2048, C::KBLK, 1024), C::IDESC_QS, (kt > 0 || ks > 0));
+                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
+                                (kt > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BN / 16; ++ks)
-                        mma_bf16_ss(tmem + C::TMEM_DQT, sw128_desc(aDst + ks * 32, 16, 1024),
-                                    sw128_desc(aKt + ks * 2048, C::KBLK, 1024), C::IDESC_QT, (kt > 0 || ks > 0));
+                        mma_bf16_ts(tmem + C::TMEM_DQT, tmem + buf * 128 + 64 + ds_col(ks), desc_add(mKt, ks * 2048),
+                                    C::IDESC_QT, (kt > 0 || ks > 0));
                 }
-                mma_commit(&bar_dsempty);
                 mma_commit(&bar_kempty[s]);
+                if (kt + 2 < n_kt && !issue_s(kt + 2)) break;
             }
             mma_commit(&bar_done);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = query)
-        // Warpgroup wg handles key columns [32 wg, 32 wg + 32) of every tile and
-        // drains its share of the dQ columns at the end.
         const int wg = (warp - 2) >> 2;
+        const int par = wg % kBwdParities, half = wg / kBwdParities;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int gq = q0 + row;
-        const int c0 = wg * 32;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        const uint32_t bufc = lane_base + par * 128;
         float Lt = 0.f, Ls = 0.f, g = 0.f, KL2 = 0.f;
         if (gq < p.N_Q) {
             const size_t r = (size_t)bh * p.N_Q + gq;
@@ -530,41 +511,37 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         }
         const int lim = p.causal ? min(p.N_K, gq + off + 1) : p.N_K;   // first hidden key
         bool ok = true;
-        for (int kt = 0; kt < n_kt; ++kt) {
-            const int buf = kt & 1, use = kt >> 1;
-            if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 26)) { ok = false; break; }
+        for (int kt = par; kt < n_kt; kt += kBwdParities) {
+            if (!mbar_wait(&bar_sfull[par], (kt >> 1) & 1, p.st, abort_v, 26)) { ok = false; break; }
             tc_fence_after();
-            const int kb = kt * C::BN + c0;
-            const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
-            uint32_t ps[16], pt[16];
-            {
+#pragma unroll
+            for (int cc = 0; cc < C::CW / 32; ++cc) {
+                const int c = half * (C::CW / 32) + cc;   // chunk of the tile
+                const int kb = kt * C::BN + c * 32;
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 128 + c0, ut);
-                tmem_ld32(lane_base + buf * 128 + 64 + c0, us);
+                tmem_ld32(bufc + c * 32, ut);
+                tmem_ld32(bufc + 64 + c * 32, us);
                 tmem_ld_wait();
+                const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
+                uint32_t ps[16], pt[16];
                 if (masked) {
 #pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        const int j = kb + k;
-                        ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Ls, g, KL2, j < lim,
-                                               j + 1 < lim, ps[k >> 1], pt[k >> 1]);
-                    }
+                    for (int k = 0; k < 32; k += 2)
+                        ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Lt, Ls, Ls, g, g,
+                                               KL2, KL2, kb + k < lim, kb + k + 1 < lim, ps[k >> 1], pt[k >> 1]);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; k += 2)
-                        ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Ls, g, KL2, true,
-                                                true, ps[k >> 1], pt[k >> 1]);
+                        ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Lt, Ls, Ls, g, g,
+                                                KL2, KL2, true, true, ps[k >> 1], pt[k >> 1]);
                 }
+                tmem_st16(bufc + c * 32, ps);
+                if (TEACHER) tmem_st16(bufc + 64 + c * 32, pt);
             }
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sempty[buf]);
-            if (kt > 0 && !mbar_wait(&bar_dsempty, (kt - 1) & 1, p.st, abort_v, 27)) { ok = false; break; }
-            store_row32(sDss, row, wg * 4, ps);
-            if (TEACHER) store_row32(sDst, row, wg * 4, pt);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull);
+            if (lane == 0) mbar_arrive(&bar_dsfull[par]);
         }
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();

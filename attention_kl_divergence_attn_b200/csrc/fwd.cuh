@@ -6,18 +6,21 @@
 // coupled two-distribution KL reduction, so neither softmax is materialised.
 //
 // One CTA owns 128 query rows of one (batch, head).  Roles (2 + 4*NWG warps):
-//   warp 0      TMA producer: Q_t, Q_s once; K_t, K_s tiles of 128 keys into
+//   warp 0      TMA producer: Q_t, Q_s once; K_t, K_s tiles of 64 keys into
 //               an NSTAGE-deep shared-memory ring.
 //   warp 1      MMA issuer (one elected thread) and TMEM owner: per key tile
 //               S_t = Q_t K_t^T and S_s = Q_s K_s^T as tcgen05.mma (bf16 in,
-//               fp32 accumulate) into one of two TMEM buffers (2 x 256 cols).
-//   warps 2..   NWG softmax warpgroups: thread = query row = TMEM lane.  Each
-//               warpgroup reads its 128/NWG key columns of both logit tiles
-//               in 32-column chunks (tcgen05.ld 32x32b) and updates its own
-//               per-row online state (M_t, l_t, A, M_s, l_s); row reductions
-//               are thread-local because the 32x32b layout gives each thread
-//               one whole row.  The warpgroups' states are merged at the end
-//               (the state is associative: rescale both to the larger max).
+//               fp32 accumulate) into one of four TMEM buffers (4 x 128 cols).
+//   warps 2..   NWG = 2 softmax warpgroups in ping-pong: warpgroup w owns key
+//               tiles w, w+2, ... and TMEM buffers w and w+2, so the MMA warp
+//               fills a warpgroup's next buffer while it works on the current
+//               one and neither warpgroup waits for its logits.  Thread = query row
+//               = TMEM lane; it reads its row of both logit tiles in 32-column
+//               chunks (tcgen05.ld 32x32b) and updates its own per-row online
+//               state (M_t, l_t, A, M_s, l_s); row reductions are thread-local
+//               because the 32x32b layout gives each thread one whole row.
+//               The warpgroups' states are merged at the end (the state is
+//               associative: rescale both to the larger maximum).
 // State (log2 units, y = scale * log2(e) * q.k):
 //   M_t, M_s  running maxima of y_t, y_s
 //   l_t = sum 2^(y_t - M_t),  l_s = sum 2^(y_s - M_s)
@@ -39,8 +42,10 @@ struct FwdParams {
 
 template <int DT, int DS, int NWG>
 struct FwdCfg {
-    static constexpr int BM = 128, BN = 128;
-    static constexpr int BLK = 128 * 128;                    // one [128 rows][64] bf16 box
+    static constexpr int BM = 128, BN = 64;                  // query rows per CTA, keys per tile
+    static constexpr int BLK = 128 * 128;                    // one [128 rows][64] bf16 box (Q)
+    static constexpr int KBLK = BN * 128;                    // one [64 rows][64] bf16 box (K)
+    static constexpr int NBUF = 4;                           // TMEM logit buffers (S_t, S_s: 64 cols each)
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int Q_BYTES = QT_BYTES + QS_BYTES;
@@ -49,10 +54,9 @@ struct FwdCfg {
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
     static constexpr int SMEM = Q_BYTES + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int THREADS = 64 + 128 * NWG;           // TMA warp, MMA warp, NWG softmax warpgroups
-    static constexpr int CW = BN / NWG;                      // key columns of a tile per warpgroup
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
-    static_assert(CW % 32 == 0, "each warpgroup reads whole 32-column chunks");
+    static_assert(NWG == 2, "two ping-pong warpgroups, two TMEM buffers each");
 };
 
 // Number of key tiles a 128-row query tile starting at q0 must visit.
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     uint8_t *sQs = sQt + C::QT_BYTES;
     uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
 
-    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_sempty[2];
+    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
@@ -135,9 +139,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             mbar_init(&bar_kfull[s], 1);
             mbar_init(&bar_kempty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4 * NWG);
+            mbar_init(&bar_sempty[b], 4);
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -169,10 +173,10 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::BLK, &mKt, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, kt * C::BN, bh);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(st + C::KT_BYTES + b * C::BLK, &mKs, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, kt * C::BN, bh);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -186,28 +190,29 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Descriptors are built once (warp-uniform) and advanced by constant
+        // offsets, so the elected thread issues one MMA every few cycles.
+        const uint64_t dQt = sw128_desc(smem_u32(sQt), 16, 1024), dQs = sw128_desc(smem_u32(sQs), 16, 1024);
+        const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);
         if (elect_one()) {
             if (mbar_wait(&bar_q, 0, p.st, abort_v, 2)) {
-                const uint32_t aQt = smem_u32(sQt), aQs = smem_u32(sQs);
                 for (int kt = 0; kt < n_kt; ++kt) {
                     const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
-                    const int buf = kt & 1, use = kt >> 1;
+                    const int buf = kt % C::NBUF, use = kt / C::NBUF;
                     if (!mbar_wait(&bar_kfull[s], n & 1, p.st, abort_v, 3)) break;
                     if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, p.st, abort_v, 4)) break;
                     tc_fence_after();
-                    const uint32_t aKt = smem_u32(sK + s * C::STAGE_BYTES), aKs = aKt + C::KT_BYTES;
-                    const uint32_t dSt = tmem + buf * 256, dSs = dSt + 128;
+                    const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES), dKs = desc_add(dKt, C::KT_BYTES);
+                    const uint32_t dSt = tmem + buf * 128, dSs = dSt + 64;
 #pragma unroll
                     for (int kk = 0; kk < DT / 16; ++kk) {
-                        const uint32_t o = (kk >> 2) * C::BLK + (kk & 3) * 32;
-                        mma_bf16_ss(dSt, sw128_desc(aQt + o, 16, 1024), sw128_desc(aKt + o, 16, 1024), C::IDESC,
-                                    kk > 0);
+                        const uint32_t oq = (kk >> 2) * C::BLK + (kk & 3) * 32, ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ss(dSt, desc_add(dQt, oq), desc_add(dKt, ok), C::IDESC, kk > 0);
                     }
 #pragma unroll
                     for (int kk = 0; kk < DS / 16; ++kk) {
-                        const uint32_t o = (kk >> 2) * C::BLK + (kk & 3) * 32;
-                        mma_bf16_ss(dSs, sw128_desc(aQs + o, 16, 1024), sw128_desc(aKs + o, 16, 1024), C::IDESC,
-                                    kk > 0);
+                        const uint32_t oq = (kk >> 2) * C::BLK + (kk & 3) * 32, ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ss(dSs, desc_add(dQs, oq), desc_add(dKs, ok), C::IDESC, kk > 0);
                     }
                     mma_commit(&bar_sfull[buf]);
                     mma_commit(&bar_kempty[s]);
@@ -215,34 +220,32 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        // Warpgroup wg reads key columns [wg*CW, (wg+1)*CW) of every tile for all 128 rows
-        // (warp w may only touch TMEM lanes 32*(w%4)..+31); the per-row states of the
-        // warpgroups are merged at the end with the associative rule of the recurrence.
+        // ------------------------------------------------------------ softmax warpgroups (ping-pong)
         const int wg = (warp - 2) >> 2;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int grow = q0 + row;
-        const int c0 = wg * C::CW;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
-        for (int kt = 0; kt < n_kt; ++kt) {
-            const int buf = kt & 1, use = kt >> 1;
-            if (!mbar_wait(&bar_sfull[buf], use & 1, p.st, abort_v, 5)) break;
+        for (int kt = wg; kt < n_kt; kt += 2) {
+            const int buf = kt % C::NBUF;
+            const uint32_t bufc = lane_base + buf * 128;
+            if (!mbar_wait(&bar_sfull[buf], (kt / C::NBUF) & 1, p.st, abort_v, 5)) break;
             tc_fence_after();
-            const int k0 = kt * C::BN + c0;
-            const bool masked = (k0 + C::CW > p.N_K) || (p.causal && (k0 + C::CW - 1 > q0 + off));
-#pragma unroll 1
-            for (int c = 0; c < C::CW / 32; ++c) {
+            const int k0 = kt * C::BN;
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+                const int kc = k0 + c * 32;
                 float ut[32], us[32];
-                tmem_ld32(lane_base + buf * 256 + c0 + c * 32, ut);
-                tmem_ld32(lane_base + buf * 256 + 128 + c0 + c * 32, us);
+                tmem_ld32(bufc + c * 32, ut);
+                tmem_ld32(bufc + 64 + c * 32, us);
                 tmem_ld_wait();
+                const bool masked = (kc + 32 > p.N_K) || (p.causal && (kc + 31 > q0 + off));
                 if (masked) {
                     const int lim = p.causal ? min(p.N_K, grow + off + 1) : p.N_K;   // first hidden key
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
-                        if (k0 + c * 32 + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }
+                        if (kc + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }
                     }
                     online_chunk<true>(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
                 } else {

@@ -253,8 +253,9 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     if ((st = check_device()) != STREAMKL_OK) return st;
 
     CUtensorMap mqt, mkt, mqs, mks;
-    if (!make_map(&mqt, q_t, d_t, N_Q, BH, 128) || !make_map(&mkt, k_t, d_t, N_K, BH, 128) ||
-        !make_map(&mqs, q_s, d_s, N_Q, BH, 128) || !make_map(&mks, k_s, d_s, N_K, BH, 128))
+    // Q boxes of 128 rows (one query tile), K boxes of 64 rows (one key tile)
+    if (!make_map(&mqt, q_t, d_t, N_Q, BH, 128) || !make_map(&mkt, k_t, d_t, N_K, BH, 64) ||
+        !make_map(&mqs, q_s, d_s, N_Q, BH, 128) || !make_map(&mks, k_s, d_s, N_K, BH, 64))
         return STREAMKL_ERR_CUDA;
     FwdParams p;
     p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
