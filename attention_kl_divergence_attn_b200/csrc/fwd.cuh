@@ -11,10 +11,11 @@
 //   warp 1      MMA issuer (one elected thread) and TMEM owner: per key tile
 //               S_t = Q_t K_t^T and S_s = Q_s K_s^T as tcgen05.mma (bf16 in,
 //               fp32 accumulate) into one of four TMEM buffers (4 x 128 cols).
-//   warps 2..   NWG = 2 softmax warpgroups in ping-pong: warpgroup w owns key
-//               tiles w, w+2, ... and TMEM buffers w and w+2, so the MMA warp
-//               fills a warpgroup's next buffer while it works on the current
-//               one and neither warpgroup waits for its logits.  Thread = query row
+//   warps 2..   4 softmax warpgroups: 2 parities in ping-pong x 2 column halves.
+//               Warpgroup (p, h) owns key tiles p, p+2, ... (TMEM buffers p and
+//               p+2, so the MMA warp fills a parity's next buffer while it works
+//               on the current one) and, of each, the 32 key columns of half h.
+//               Four warps per SM sub-partition keep the ex2 unit fed.  Thread = query row
 //               = TMEM lane; it reads its row of both logit tiles in 32-column
 //               chunks (tcgen05.ld 32x32b) and updates its own per-row online
 //               state (M_t, l_t, A, M_s, l_s); row reductions are thread-local
@@ -53,10 +54,12 @@ struct FwdCfg {
     static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
     static constexpr int SMEM = Q_BYTES + NSTAGE * STAGE_BYTES + 1024;
+    static constexpr int NH = NWG / 2;                       // column halves per parity
+    static constexpr int CW = BN / NH;                       // key columns per warpgroup and tile
     static constexpr int THREADS = 64 + 128 * NWG;           // TMA warp, MMA warp, NWG softmax warpgroups
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
-    static_assert(NWG == 2, "two ping-pong warpgroups, two TMEM buffers each");
+    static_assert(NWG == 2 || NWG == 4, "2 parities x NWG/2 column halves");
 };
 
 // Number of key tiles a 128-row query tile starting at q0 must visit.
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         }
         for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_sempty[b], 4);
+            mbar_init(&bar_sempty[b], 4 * C::NH);
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -222,19 +225,21 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     } else {
         // ------------------------------------------------------------ softmax warpgroups (ping-pong)
         const int wg = (warp - 2) >> 2;
+        const int par = wg & 1, half = wg >> 1;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const int grow = q0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
-        for (int kt = wg; kt < n_kt; kt += 2) {
+        for (int kt = par; kt < n_kt; kt += 2) {
             const int buf = kt % C::NBUF;
             const uint32_t bufc = lane_base + buf * 128;
             if (!mbar_wait(&bar_sfull[buf], (kt / C::NBUF) & 1, p.st, abort_v, 5)) break;
             tc_fence_after();
             const int k0 = kt * C::BN;
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
+            for (int cc = 0; cc < C::CW / 32; ++cc) {
+                const int c = half * (C::CW / 32) + cc;
                 const int kc = k0 + c * 32;
                 float ut[32], us[32];
                 tmem_ld32(bufc + c * 32, ut);

@@ -82,7 +82,7 @@ cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-constexpr int kFwdWarpgroups = 2;
+constexpr int kFwdWarpgroups = 4;
 
 template <int DT, int DS>
 streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const CUtensorMap &qs,
