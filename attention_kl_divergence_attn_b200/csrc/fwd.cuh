@@ -72,10 +72,11 @@ __device__ __forceinline__ int fwd_key_tiles(int q0, int N_Q, int N_K, int causa
     return (kend + BN - 1) / BN;
 }
 
-// Online update with one 32-column chunk of raw logits (u = q.k, unscaled).
-template <bool MASKED>
-__device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
-                                             float &Ms, float &lt, float &ls, float &A) {
+// Online update with one 32-column chunk of raw logits (u = q.k, unscaled),
+// scalar form used for chunks that contain masked (hidden or padding) keys,
+// which are passed in as -inf.
+__device__ __forceinline__ void online_chunk_masked(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
+                                                    float &Ms, float &lt, float &ls, float &A) {
     float m0 = fmaxf(ut[0], ut[1]), m1 = fmaxf(ut[2], ut[3]);
     float n0 = fmaxf(us[0], us[1]), n1 = fmaxf(us[2], us[3]);
 #pragma unroll
@@ -87,7 +88,7 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
     }
     const float Mt_new = fmaxf(Mt, fmaxf(m0, m1) * ct);
     const float Ms_new = fmaxf(Ms, fmaxf(n0, n1) * cs);
-    if (MASKED && Mt_new == -INFINITY) return;      // nothing visible so far
+    if (Mt_new == -INFINITY) return;      // nothing visible so far
     const float at = ex2(Mt - Mt_new), as = ex2(Ms - Ms_new);
     float st[4] = {0.f, 0.f, 0.f, 0.f}, ss[4] = {0.f, 0.f, 0.f, 0.f}, sa[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -97,8 +98,7 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
         const float et = ex2(xt), es = ex2(xs);
         st[k & 3] += et;
         ss[k & 3] += es;
-        float dx = xt - xs;
-        if (MASKED) dx = (ut[k] == -INFINITY) ? 0.f : dx;
+        const float dx = (ut[k] == -INFINITY) ? 0.f : xt - xs;
         sa[k & 3] = fmaf(et, dx, sa[k & 3]);
     }
     const float sum_t = (st[0] + st[1]) + (st[2] + st[3]);
@@ -107,6 +107,48 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
     lt = fmaf(lt, at, sum_t);
     ls = fmaf(ls, as, sum_s);
     A = fmaf(A, at, fmaf(Mt_new - Ms_new, sum_t, sum_a));
+    Mt = Mt_new;
+    Ms = Ms_new;
+}
+
+// The same update for a fully visible chunk, on packed fp32 pairs: the
+// element-wise work issues one instruction per two keys, the chunk maxima use
+// three-input max, and a quarter of the exponentials (every second pair of
+// student terms) is evaluated on the FMA pipe by exp2_poly2<5> so that the ex2
+// unit is not the only resource doing exponentials.
+__device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
+                                             float &Ms, float &lt, float &ls, float &A) {
+    float m0 = fmax3(ut[0], ut[1], ut[2]), m1 = fmax3(ut[3], ut[4], ut[5]);
+    float n0 = fmax3(us[0], us[1], us[2]), n1 = fmax3(us[3], us[4], us[5]);
+#pragma unroll
+    for (int k = 6; k < 30; k += 4) {
+        m0 = fmax3(m0, ut[k], ut[k + 1]);
+        m1 = fmax3(m1, ut[k + 2], ut[k + 3]);
+        n0 = fmax3(n0, us[k], us[k + 1]);
+        n1 = fmax3(n1, us[k + 2], us[k + 3]);
+    }
+    const float Mt_new = fmaxf(Mt, fmax3(m0, m1, fmaxf(ut[30], ut[31])) * ct);
+    const float Ms_new = fmaxf(Ms, fmax3(n0, n1, fmaxf(us[30], us[31])) * cs);
+    const float at = ex2(Mt - Mt_new), as = ex2(Ms - Ms_new);
+    const uint64_t ct2 = f2splat(ct), cs2 = f2splat(cs);
+    const uint64_t nMt = f2splat(-Mt_new), nMs = f2splat(-Ms_new);
+    uint64_t st[2] = {0ull, 0ull}, ss[2] = {0ull, 0ull}, sa[2] = {0ull, 0ull};
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+        const int j = (k >> 1) & 1;
+        const uint64_t xt = f2fma(f2pack(ut[k], ut[k + 1]), ct2, nMt);
+        const uint64_t xs = f2fma(f2pack(us[k], us[k + 1]), cs2, nMs);
+        const uint64_t et = ex2_pair(xt);
+        const uint64_t es = j ? exp2_poly2<5>(xs) : ex2_pair(xs);
+        st[j] = f2add(st[j], et);
+        ss[j] = f2add(ss[j], es);
+        sa[j] = f2fma(et, f2sub(xt, xs), sa[j]);
+    }
+    const float2 t2 = f2unpack(f2add(st[0], st[1])), s2 = f2unpack(f2add(ss[0], ss[1]));
+    const float2 a2 = f2unpack(f2add(sa[0], sa[1]));
+    lt = fmaf(lt, at, t2.x + t2.y);
+    ls = fmaf(ls, as, s2.x + s2.y);
+    A = fmaf(A, at, fmaf(Mt_new - Ms_new, t2.x + t2.y, a2.x + a2.y));
     Mt = Mt_new;
     Ms = Ms_new;
 }
@@ -252,9 +294,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                     for (int k = 0; k < 32; ++k) {
                         if (kc + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }
                     }
-                    online_chunk<true>(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                    online_chunk_masked(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
                 } else {
-                    online_chunk<false>(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                    online_chunk(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
                 }
             }
             tc_fence_before();
