@@ -293,26 +293,42 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
 #pragma unroll
             for (int cc = 0; cc < C::CW / 32; ++cc) {
                 const int c = half * (C::CW / 32) + cc;   // chunk of the tile
-                float ut[32], us[32];
-                tmem_ld32(bufc + c * 32, ut);
-                tmem_ld32(bufc + 64 + c * 32, us);
-                tmem_ld_wait();
                 const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c * 32 + off);
-                uint32_t ps[16], pt[16];
+                // Two 16-column pieces per chunk: each piece loads its logits, computes
+                // dS with the mask test hoisted out of the element loop (so the compiler
+                // interleaves the independent pairs) and stores its 8 packed dS columns
+                // over columns of this chunk that the first piece has already read.
 #pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const int q = c * 32 + k;
-                    const float4 e0 = cst[q], e1 = cst[q + 1];
-                    if (masked)
-                        ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y, e1.y,
-                                               e0.z, e1.z, e0.w, e1.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
-                    else
-                        ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
-                                                e1.y, e0.z, e1.z, e0.w, e1.w, true, true, ps[k >> 1], pt[k >> 1]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float ut[16], us[16];
+                    tmem_ld16(bufc + c * 32 + hh * 16, ut);
+                    tmem_ld16(bufc + 64 + c * 32 + hh * 16, us);
+                    tmem_ld_wait();
+                    uint32_t ps[8], pt[8];
+                    if (masked) {
+#pragma unroll
+                        for (int k = 0; k < 16; k += 2) {
+                            if (k == 8) asm volatile("" ::: "memory");   // bound the constants in flight
+                            const int q = c * 32 + hh * 16 + k;
+                            const float4 e0 = cst[q], e1 = cst[q + 1];
+                            ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
+                                                   e1.y, e0.z, e1.z, e0.w, e1.w, q >= qmin, q + 1 >= qmin, ps[k >> 1],
+                                                   pt[k >> 1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; k += 2) {
+                            if (k == 8) asm volatile("" ::: "memory");
+                            const int q = c * 32 + hh * 16 + k;
+                            const float4 e0 = cst[q], e1 = cst[q + 1];
+                            ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
+                                                    e1.y, e0.z, e1.z, e0.w, e1.w, true, true, ps[k >> 1], pt[k >> 1]);
+                        }
+                    }
+                    // piece hh writes columns [8 hh, 8 hh + 8) of the chunk, which piece 0 read
+                    tmem_st8(bufc + c * 32 + hh * 8, ps);
+                    if (TEACHER) tmem_st8(bufc + 64 + c * 32 + hh * 8, pt);
                 }
-                // the columns written here were read by this chunk's (already completed) loads
-                tmem_st16(bufc + c * 32, ps);
-                if (TEACHER) tmem_st16(bufc + 64 + c * 32, pt);
             }
             tmem_st_wait();
             tc_fence_before();
