@@ -183,10 +183,35 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
         }
+        // Per-query constants of a tile: lane l handles queries l and l + 32.  They
+        // are fetched from global memory two tiles ahead into registers, with loads
+        // the compiler may not move (ld_now), so that their latency overlaps the
+        // tiles in between instead of stalling the ring.
+        auto load_consts = [&](int t, float4 (&v)[2]) {
+            const int q0 = (first_qt + t) * C::BM;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = q0 + lane + 32 * h;
+                v[h] = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
+                if (t < n_qt && i < p.N_Q) {
+                    const size_t r = (size_t)bh * p.N_Q + i;
+                    v[h].x = ld_now(p.lse_t + r);
+                    v[h].y = ld_now(p.lse_s + r);
+                    v[h].z = p.dkl ? ld_now(p.dkl + r) : p.g_const;
+                    v[h].w = ld_now(p.kl + r);
+                }
+            }
+        };
+        float4 c0[2], c1[2], c2[2];
+        load_consts(0, c1);
+        load_consts(1, c2);
         int issued = 0;
         for (int t = 0; t < n_qt; ++t) {
             const int s = t % C::NSTAGE, n = t / C::NSTAGE;
             const int q0 = (first_qt + t) * C::BM;
+            c0[0] = c1[0]; c0[1] = c1[1];
+            c1[0] = c2[0]; c1[1] = c2[1];
+            load_consts(t + 2, c2);
             if (n > 0 && !mbar_wait(&bar_qempty[s], (n - 1) & 1, p.st, abort_v, 11)) break;
             uint8_t *st = sQ + s * C::STAGE_BYTES;
             if (lane == 0) {
@@ -200,19 +225,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             }
             float4 *cst = reinterpret_cast<float4 *>(st + C::STAGE_TMA);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int q = lane + 32 * h;
-                const int i = q0 + q;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
-                if (i < p.N_Q) {
-                    const size_t r = (size_t)bh * p.N_Q + i;
-                    v.x = p.lse_t[r] * kLog2eF;
-                    v.y = p.lse_s[r] * kLog2eF;
-                    v.z = p.dkl ? p.dkl[r] : p.g_const;
-                    v.w = p.kl[r] * kLog2eF;
-                }
-                cst[q] = v;
-            }
+            for (int h = 0; h < 2; ++h)
+                cst[lane + 32 * h] = make_float4(c0[h].x * kLog2eF, c0[h].y * kLog2eF, c0[h].z, c0[h].w * kLog2eF);
             mbar_arrive(&bar_qfull[s]);
             issued = t + 1;
         }
