@@ -17,8 +17,13 @@
 // deterministic result):
 //   streamkl_bwd_dkv_kernel  CTA = 128 keys of one head; loops over 64-query
 //       tiles: S^T = K Q^T (teacher and student), dS^T, dK += dS^T Q.
-//       Thread = key row; per-query constants come from a small shared-memory
-//       table the producer warp fills next to each TMA tile of Q.
+//       Thread = key row, so the per-query log-sum-exps would be a per-element
+//       shared-memory load; instead one extra rank-1 MMA per tensor and tile
+//       adds them to the logits: A = a constant [128 x 16] matrix whose rows
+//       are (1, 1, 1, 0, ...), B = the tile's rows (h, m, l, 0, ...) with
+//       h + m + l = -LSE / scale split into three bf16 terms (about fp32
+//       precision), so the accumulator holds q.k - LSE / scale directly.
+//       Only g and KL per query come from a small shared-memory table.
 //   streamkl_bwd_dq_kernel   CTA = 128 queries of one head; loops over 64-key
 //       tiles: S = Q K^T, dS, dQ += dS K.  Thread = query row; per-row
 //       constants live in registers.
@@ -39,6 +44,8 @@
 // tile t+2 can be issued into buffer t & 1 right after the gradient MMA of t.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "sm100.cuh"
 
 namespace skl {
@@ -49,11 +56,25 @@ struct BwdParams {
     float out_t, out_s;           // output scales: scale_t * ln2 (teacher), scale_s (student)
     const float *kl, *lse_t, *lse_s, *dkl;
     float g_const;                // g when dkl == nullptr
+    float inv_scale_t, inv_scale_s;
     float *dq_s, *dq_t, *dk_s, *dk_t;
     DevStatus st;
 };
 
 constexpr float kLog2eF = 1.4426950408889634074f;
+
+// x as three bf16 values h + m + l (each the rounding of what is left), packed
+// as K elements 0..2 of a bf16 row (lower half first); the sum reproduces x to
+// about 2^-24 relative, so a rank-1 MMA can add an fp32-accurate per-column
+// offset to an accumulator.
+__device__ __forceinline__ uint2 split3_bf16(float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+    return make_uint2((uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(m) << 16),
+                      (uint32_t)__bfloat16_as_ushort(l));
+}
 
 // dS for two adjacent elements, packed as bf16x2 (lower half = first element).
 // Per-element constants: L (log2-domain LSEs), g and KL*log2(e).
@@ -108,10 +129,13 @@ struct DkvCfg {
     static constexpr int QBLK = 64 * 128;          // [64 rows][64] bf16 box
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
-    static constexpr int CONST_BYTES = BM * 16;   // float4 per query
     static constexpr int STAGE_TMA = QT_BYTES + QS_BYTES;
-    static constexpr int STAGE_BYTES = STAGE_TMA + CONST_BYTES;
-    static constexpr int FIXED = KT_BYTES + KS_BYTES;
+    static constexpr int BIAS_BYTES = BM * 16 * 2;  // [64 queries][16] bf16, unswizzled K-major
+    static constexpr int GK_BYTES = BM * 8;         // float2 {g, KL log2(e)} per query
+    static constexpr int BIAS_T = STAGE_TMA, BIAS_S = BIAS_T + BIAS_BYTES, GK = BIAS_S + BIAS_BYTES;
+    static constexpr int STAGE_BYTES = ((GK + GK_BYTES + 1023) / 1024) * 1024;
+    static constexpr int ONES_BYTES = BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
+    static constexpr int FIXED = KT_BYTES + KS_BYTES + ONES_BYTES;
     static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
@@ -133,7 +157,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sKt = smem;
     uint8_t *sKs = sKt + C::KT_BYTES;
-    uint8_t *sQ = sKs + C::KS_BYTES;               // stages: Q_t, Q_s, per-query constants
+    uint8_t *sOnes = sKs + C::KS_BYTES;            // rank-1 MMA operand (1, 1, 1, 0, ...)
+    uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
 
     __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
     __shared__ uint64_t bar_done;
@@ -167,6 +192,19 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         tmem_alloc(&tmem_base_sh, 512);
         tmem_relinquish();
     }
+    // Unswizzled K-major [rows][16] bf16 layout: row r, K block kb at
+    // (r / 8) * 256 + kb * 128 + (r % 8) * 16.  The ones matrix has 1.0 in K
+    // elements 0..2 of every row; the bias tiles start all zero and the producer
+    // later writes only K elements 0..2 of each row.
+    for (int i = threadIdx.x; i < C::ONES_BYTES / 16; i += blockDim.x) {
+        const bool first_block = ((i >> 3) & 1) == 0;   // 16-byte units: 8 rows per K block
+        *reinterpret_cast<uint4 *>(sOnes + i * 16) =
+            first_block ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int st = 0; st < C::NSTAGE; ++st)
+        for (int i = threadIdx.x; i < 2 * C::BIAS_BYTES / 16; i += blockDim.x)
+            *reinterpret_cast<uint4 *>(sQ + st * C::STAGE_BYTES + C::BIAS_T + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -187,7 +225,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         // are fetched from global memory two tiles ahead into registers, with loads
         // the compiler may not move (ld_now), so that their latency overlaps the
         // tiles in between instead of stalling the ring.
-        auto load_consts = [&](int t, float4 (&v)[2]) {
+        auto load_consts = [&](int t, float4 (&v)[2]) {   // raw {lse_t, lse_s, g, kl}
             const int q0 = (first_qt + t) * C::BM;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -223,10 +261,16 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh);
             }
-            float4 *cst = reinterpret_cast<float4 *>(st + C::STAGE_TMA);
+            float2 *gk = reinterpret_cast<float2 *>(st + C::GK);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-                cst[lane + 32 * h] = make_float4(c0[h].x * kLog2eF, c0[h].y * kLog2eF, c0[h].z, c0[h].w * kLog2eF);
+            for (int h = 0; h < 2; ++h) {
+                const int q = lane + 32 * h;
+                gk[q] = make_float2(c0[h].z, c0[h].w * kLog2eF);
+                const uint32_t row = (uint32_t)(q >> 3) * 256u + (uint32_t)(q & 7) * 16u;
+                *reinterpret_cast<uint2 *>(st + C::BIAS_T + row) = split3_bf16(-c0[h].x * p.inv_scale_t);
+                *reinterpret_cast<uint2 *>(st + C::BIAS_S + row) = split3_bf16(-c0[h].y * p.inv_scale_s);
+            }
+            fence_proxy_async_smem();          // the bias rows are read by the tensor core
             mbar_arrive(&bar_qfull[s]);
             issued = t + 1;
         }
@@ -244,21 +288,26 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dKt = sw128_desc(smem_u32(sKt), 16, 1024), dKs = sw128_desc(smem_u32(sKs), 16, 1024);
         const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);          // K-major view of a stage
         const uint64_t dQ0mn = sw128_desc(smem_u32(sQ), C::QBLK, 1024);   // MN-major view of a stage
+        const uint64_t dOnes = plain_desc(smem_u32(sOnes), 128, 256);
+        const uint64_t dBias0 = plain_desc(smem_u32(sQ + C::BIAS_T), 128, 256);
         if (elect_one()) {
-            // S^T of tile t into buffer t & 1
+            // S^T of tile t into buffer t & 1, each plus its rank-1 bias -LSE / scale
             auto issue_s = [&](int t) -> bool {
                 const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
                 if (!mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 12)) return false;
                 tc_fence_after();
                 const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES), dQs = desc_add(dQt, C::QT_BYTES);
+                const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES), dBs = desc_add(dBt, C::BIAS_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DT / 16; ++kk)
                     mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32),
                                 desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk)
                     mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32),
                                 desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                mma_bf16_ss(tmem + buf * 128 + 64, dOnes, dBs, C::IDESC_S, 1);
                 mma_commit(&bar_sfull[buf]);
                 return true;
             };
@@ -302,7 +351,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             if (!mbar_wait(&bar_sfull[par], (t >> 1) & 1, p.st, abort_v, 16) ||
                 !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
             tc_fence_after();
-            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::STAGE_TMA);
+            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::GK);   // {g,K,g',K'}
             const int qmin = gk - off - q0;        // first visible query column (causal)
 #pragma unroll
             for (int cc = 0; cc < C::CW / 32; ++cc) {
@@ -324,19 +373,18 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                         for (int k = 0; k < 16; k += 2) {
                             if (k == 8) asm volatile("" ::: "memory");   // bound the constants in flight
                             const int q = c * 32 + hh * 16 + k;
-                            const float4 e0 = cst[q], e1 = cst[q + 1];
-                            ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
-                                                   e1.y, e0.z, e1.z, e0.w, e1.w, q >= qmin, q + 1 >= qmin, ps[k >> 1],
-                                                   pt[k >> 1]);
+                            const float4 e = cst[q >> 1];
+                            ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, 0.f, 0.f, 0.f, 0.f,
+                                                   e.x, e.z, e.y, e.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
                         }
                     } else {
 #pragma unroll
                         for (int k = 0; k < 16; k += 2) {
                             if (k == 8) asm volatile("" ::: "memory");
                             const int q = c * 32 + hh * 16 + k;
-                            const float4 e0 = cst[q], e1 = cst[q + 1];
-                            ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, e0.x, e1.x, e0.y,
-                                                    e1.y, e0.z, e1.z, e0.w, e1.w, true, true, ps[k >> 1], pt[k >> 1]);
+                            const float4 e = cst[q >> 1];
+                            ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, 0.f, 0.f, 0.f, 0.f,
+                                                    e.x, e.z, e.y, e.w, true, true, ps[k >> 1], pt[k >> 1]);
                         }
                     }
                     // piece hh writes columns [8 hh, 8 hh + 8) of the chunk, which piece 0 read

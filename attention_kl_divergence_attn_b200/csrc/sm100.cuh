@@ -246,6 +246,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo,
     return d;
 }
 
+// Shared-memory matrix descriptor of tcgen05.mma for an unswizzled K-major
+// operand of 16-element rows: 8-row x 16-byte core matrices, `lbo` bytes between
+// the two core matrices of a row block (K elements 0-7 and 8-15), `sbo` bytes
+// between 8-row blocks.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;                 // descriptor version (sm_100), no swizzle
+    return d;
+}
+
 // A descriptor advanced by `bytes` (a multiple of 16): the start address lives in
 // the low 14 bits in 16-byte units, and shared-memory addresses stay below 256 KB,
 // so the add never carries into the other fields.

@@ -183,6 +183,8 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     p.out_s = scale_s;
     p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s; p.dkl = dkl;
     p.g_const = (float)((double)dloss / ((double)BH * (double)N_Q));
+    p.inv_scale_t = 1.0f / scale_t;
+    p.inv_scale_s = 1.0f / scale_s;
     p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
     p.st.word = static_cast<uint32_t *>(workspace);
     p.st.budget_ns = kWaitBudgetNs;
