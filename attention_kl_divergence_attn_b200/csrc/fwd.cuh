@@ -112,10 +112,10 @@ __device__ __forceinline__ void online_chunk_masked(float (&ut)[32], float (&us)
 }
 
 // The same update for a fully visible chunk, on packed fp32 pairs: the
-// element-wise work issues one instruction per two keys, the chunk maxima use
-// three-input max, and a quarter of the exponentials (every second pair of
-// student terms) is evaluated on the FMA pipe by exp2_poly2<5> so that the ex2
-// unit is not the only resource doing exponentials.
+// element-wise work issues one instruction per two keys and the chunk maxima
+// use three-input max.  (Moving part of the exponentials to the FMA pipe with a
+// polynomial was measured slower here: the loop is bound by ex2 and issue
+// slots together, so the extra instructions cost more than the ex2 time saved.)
 __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
                                              float &Ms, float &lt, float &ls, float &A) {
     float m0 = fmax3(ut[0], ut[1], ut[2]), m1 = fmax3(ut[3], ut[4], ut[5]);
@@ -139,7 +139,7 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
         const uint64_t xt = f2fma(f2pack(ut[k], ut[k + 1]), ct2, nMt);
         const uint64_t xs = f2fma(f2pack(us[k], us[k + 1]), cs2, nMs);
         const uint64_t et = ex2_pair(xt);
-        const uint64_t es = j ? exp2_poly2<5>(xs) : ex2_pair(xs);
+        const uint64_t es = ex2_pair(xs);
         st[j] = f2add(st[j], et);
         ss[j] = f2add(ss[j], es);
         sa[j] = f2fma(et, f2sub(xt, xs), sa[j]);

@@ -338,43 +338,6 @@ __device__ __forceinline__ uint64_t ex2_pair(uint64_t x) {
     return f2pack(ex2(v.x), ex2(v.y));
 }
 
-// 2^x of both halves on the FMA pipe, leaving the ex2 unit free for other
-// elements.  Range reduction x = n + f, n = rint(x): adding 1.5 * 2^23 rounds x
-// to an integer held in the low mantissa bits, so subtracting it back gives n
-// exactly and f = x - n lies in [-1/2, 1/2].  2^f comes from a polynomial whose
-// coefficients minimise the maximum relative error on that interval (fitted
-// by csrc/exp2_poly_fit.py: degree 3 -> 7.5e-5, degree 5 -> 2.2e-7), and 2^n is
-// applied by adding n to the exponent field (n << 23 is the low bits of the
-// rounded value shifted into place).  Inputs below -125 are clamped so the
-// result stays a normal number (2^-125 stands in for anything smaller).
-template <int DEG>
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-    static_assert(DEG == 3 || DEG == 5, "fitted degrees");
-    float2 v = f2unpack(x);
-    v.x = fmaxf(v.x, -125.f);
-    v.y = fmaxf(v.y, -125.f);
-    const uint64_t xc = f2pack(v.x, v.y);
-    const uint64_t magic = f2splat(12582912.0f);
-    const uint64_t fi = f2add(xc, magic);
-    const uint64_t f = f2sub(xc, f2sub(fi, magic));
-    uint64_t p;
-    if (DEG == 3) {
-        p = f2fma(f2splat(5.517137796e-02f), f, f2splat(2.426112145e-01f));
-        p = f2fma(p, f, f2splat(6.932610273e-01f));
-        p = f2fma(p, f, f2splat(9.999280572e-01f));
-    } else {
-        p = f2fma(f2splat(1.327647245e-03f), f, f2splat(9.675547481e-03f));
-        p = f2fma(p, f, f2splat(5.550713465e-02f));
-        p = f2fma(p, f, f2splat(2.402212024e-01f));
-        p = f2fma(p, f, f2splat(6.931469440e-01f));
-        p = f2fma(p, f, f2splat(1.000000119e+00f));
-    }
-    const float2 pf = f2unpack(p), nf = f2unpack(fi);
-    const uint32_t b0 = __float_as_uint(pf.x) + (__float_as_uint(nf.x) << 23);
-    const uint32_t b1 = __float_as_uint(pf.y) + (__float_as_uint(nf.y) << 23);
-    return f2pack(__uint_as_float(b0), __uint_as_float(b1));
-}
-
 // Byte offset of element (row, col) in a [rows][64] bf16 tile stored with the
 // 128-byte swizzle that TMA (CU_TENSOR_MAP_SWIZZLE_128B) and tcgen05 share:
 // the 16-byte chunk index is XORed with (row mod 8).  Tile base 1024-aligned.

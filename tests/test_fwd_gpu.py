@@ -55,10 +55,7 @@ def test_fwd_self_kl_is_zero():
     qt, kt = cuda(*inputs.make_inputs(w)[:2])
     kl, lt, ls, _ = streamkl_fwd(qt, kt, qt, kt, 0.1, 0.1, True)
     assert float(kl.abs().max()) < 1e-5
-    # teacher and student exponentials are evaluated by different units (part of
-    # the student terms by a polynomial with relative error <= 2.2e-7), so the
-    # two log-sum-exps agree to fp32 rounding rather than bit for bit
-    assert torch.allclose(lt, ls, rtol=1e-6, atol=1e-6)
+    assert torch.equal(lt, ls)           # teacher and student take identical paths
 
 
 def test_fwd_deterministic():
