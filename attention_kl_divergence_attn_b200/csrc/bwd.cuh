@@ -94,6 +94,88 @@ __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float u
     if (TEACHER) pt = pack_bf16((g0 * P0) * ((at0 - as0) - K0), (g1 * P1) * ((at1 - as1) - K1));
 }
 
+// The two chunk routines below turn one 32-column chunk of a warpgroup's S
+// columns (teacher logits at `at`, student at `as`) into this thread's 32 dS
+// values, written as 16 packed bf16 columns over the first half of the chunk
+// (student dS over the teacher logits, teacher dS over the student logits).
+// The logits are read in pieces of PW columns and each piece's load is issued
+// before the previous piece is computed, so the tensor-memory latency overlaps
+// the arithmetic; the stores of piece p land on columns [p PW/2, (p+1) PW/2),
+// which pieces 0..p have already read, and never on the piece in flight.
+constexpr int kBwdPiece = 8;
+
+// Query-owner chunk (thread = query row; constants per row, keys kb .. kb+31,
+// keys >= lim hidden).
+template <bool TEACHER, bool MASKED, int PW = kBwdPiece>
+__device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, float cs, float Lt, float Ls, float g,
+                                         float KL2, int kb, int lim) {
+    constexpr int NP = 32 / PW;
+    float ut[2][PW], us[2][PW];
+    tmem_ld<PW>(at, ut[0]);
+    tmem_ld<PW>(as, us[0]);
+    tmem_ld_wait_bind(ut[0], us[0]);
+#pragma unroll
+    for (int pc = 0; pc < NP; ++pc) {
+        const int cur = pc & 1;
+        if (pc + 1 < NP) {
+            tmem_ld<PW>(at + PW * (pc + 1), ut[cur ^ 1]);
+            tmem_ld<PW>(as + PW * (pc + 1), us[cur ^ 1]);
+        }
+        uint32_t ps[PW / 2], pt[PW / 2];
+#pragma unroll
+        for (int k = 0; k < PW; k += 2) {
+            const int j = kb + PW * pc + k;
+            ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, Lt, Lt, Ls, Ls,
+                                     g, g, KL2, KL2, j < lim, j + 1 < lim, ps[k >> 1], pt[k >> 1]);
+        }
+        if constexpr (PW == 8) {
+            tmem_st4(at + 4 * pc, ps);
+            if (TEACHER) tmem_st4(as + 4 * pc, pt);
+        } else {
+            tmem_st8(at + 8 * pc, ps);
+            if (TEACHER) tmem_st8(as + 8 * pc, pt);
+        }
+        if (pc + 1 < NP) tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
+    }
+}
+
+// Key-owner chunk (thread = key row; the logits already carry -LSE / scale, so
+// only g and KL log2(e) per query column come from `cst`, two queries per
+// float4 {g, K, g', K'}; columns q < qmin, relative to the chunk, are hidden).
+template <bool TEACHER, bool MASKED, int PW = kBwdPiece>
+__device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float4 *cst,
+                                          int qmin) {
+    constexpr int NP = 32 / PW;
+    float ut[2][PW], us[2][PW];
+    tmem_ld<PW>(at, ut[0]);
+    tmem_ld<PW>(as, us[0]);
+    tmem_ld_wait_bind(ut[0], us[0]);
+#pragma unroll
+    for (int pc = 0; pc < NP; ++pc) {
+        const int cur = pc & 1;
+        if (pc + 1 < NP) {
+            tmem_ld<PW>(at + PW * (pc + 1), ut[cur ^ 1]);
+            tmem_ld<PW>(as + PW * (pc + 1), us[cur ^ 1]);
+        }
+        uint32_t ps[PW / 2], pt[PW / 2];
+#pragma unroll
+        for (int k = 0; k < PW; k += 2) {
+            const int q = PW * pc + k;
+            const float4 e = cst[q >> 1];
+            ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f, 0.f,
+                                     0.f, e.x, e.z, e.y, e.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
+        }
+        if constexpr (PW == 8) {
+            tmem_st4(at + 4 * pc, ps);
+            if (TEACHER) tmem_st4(as + 4 * pc, pt);
+        } else {
+            tmem_st8(at + 8 * pc, ps);
+            if (TEACHER) tmem_st8(as + 8 * pc, pt);
+        }
+        if (pc + 1 < NP) tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
+    }
+}
+
 // Reads `NCOLS` (a multiple of 16) fp32 accumulator columns of this thread's
 // TMEM lane, scales them and writes them to dst (one row, contiguous) if `store`.
 template <int NCOLS>
@@ -357,40 +439,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             for (int cc = 0; cc < C::CW / 32; ++cc) {
                 const int c = half * (C::CW / 32) + cc;   // chunk of the tile
                 const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c * 32 + off);
-                // Two 16-column pieces per chunk: each piece loads its logits, computes
-                // dS with the mask test hoisted out of the element loop (so the compiler
-                // interleaves the independent pairs) and stores its 8 packed dS columns
-                // over columns of this chunk that the first piece has already read.
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float ut[16], us[16];
-                    tmem_ld16(bufc + c * 32 + hh * 16, ut);
-                    tmem_ld16(bufc + 64 + c * 32 + hh * 16, us);
-                    tmem_ld_wait();
-                    uint32_t ps[8], pt[8];
-                    if (masked) {
-#pragma unroll
-                        for (int k = 0; k < 16; k += 2) {
-                            if (k == 8) asm volatile("" ::: "memory");   // bound the constants in flight
-                            const int q = c * 32 + hh * 16 + k;
-                            const float4 e = cst[q >> 1];
-                            ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, 0.f, 0.f, 0.f, 0.f,
-                                                   e.x, e.z, e.y, e.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; k += 2) {
-                            if (k == 8) asm volatile("" ::: "memory");
-                            const int q = c * 32 + hh * 16 + k;
-                            const float4 e = cst[q >> 1];
-                            ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, 0.f, 0.f, 0.f, 0.f,
-                                                    e.x, e.z, e.y, e.w, true, true, ps[k >> 1], pt[k >> 1]);
-                        }
-                    }
-                    // piece hh writes columns [8 hh, 8 hh + 8) of the chunk, which piece 0 read
-                    tmem_st8(bufc + c * 32 + hh * 8, ps);
-                    if (TEACHER) tmem_st8(bufc + 64 + c * 32 + hh * 8, pt);
-                }
+                if (masked)
+                    dkv_chunk<TEACHER, true>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, cst + c * 16, qmin - c * 32);
+                else
+                    dkv_chunk<TEACHER, false>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, cst + c * 16, 0);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -596,25 +648,11 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             for (int cc = 0; cc < C::CW / 32; ++cc) {
                 const int c = half * (C::CW / 32) + cc;   // chunk of the tile
                 const int kb = kt * C::BN + c * 32;
-                float ut[32], us[32];
-                tmem_ld32(bufc + c * 32, ut);
-                tmem_ld32(bufc + 64 + c * 32, us);
-                tmem_ld_wait();
                 const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
-                uint32_t ps[16], pt[16];
-                if (masked) {
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2)
-                        ds_pair<TEACHER, true>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Lt, Ls, Ls, g, g,
-                                               KL2, KL2, kb + k < lim, kb + k + 1 < lim, ps[k >> 1], pt[k >> 1]);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2)
-                        ds_pair<TEACHER, false>(ut[k], ut[k + 1], us[k], us[k + 1], p.ct, p.cs, Lt, Lt, Ls, Ls, g, g,
-                                                KL2, KL2, true, true, ps[k >> 1], pt[k >> 1]);
-                }
-                tmem_st16(bufc + c * 32, ps);
-                if (TEACHER) tmem_st16(bufc + 64 + c * 32, pt);
+                if (masked)
+                    dq_chunk<TEACHER, true>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
+                else
+                    dq_chunk<TEACHER, false>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
             }
             tmem_st_wait();
             tc_fence_before();

@@ -344,19 +344,47 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     }
 }
 
-// Deterministic mean of n per-row values (one CTA, fp64 partial sums).
-__global__ void __launch_bounds__(1024) streamkl_mean_kernel(const float *__restrict__ v, long long n,
-                                                             float *__restrict__ out) {
-    __shared__ double red[1024];
+// Deterministic mean of n per-row values: one CTA of kMeanThreads threads,
+// each summing a fixed strided subset in fp64 (16-byte loads, eight in flight
+// per thread when the array is 16-byte aligned), then a fixed-shape tree
+// (warp shuffles, then one warp over the warp sums).  The order of additions
+// depends only on n, so the result is the same run to run.
+constexpr int kMeanThreads = 1024;
+
+__global__ void __launch_bounds__(kMeanThreads) streamkl_mean_kernel(const float *__restrict__ v, long long n,
+                                                                     float *__restrict__ out) {
+    __shared__ double red[kMeanThreads / 32];
     double s = 0.0;
-    for (long long k = threadIdx.x; k < n; k += blockDim.x) s += (double)v[k];
-    red[threadIdx.x] = s;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-        if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-        __syncthreads();
+    long long done = 0;
+    if ((reinterpret_cast<uintptr_t>(v) & 15) == 0) {
+        const float4 *v4 = reinterpret_cast<const float4 *>(v);
+        const long long n4 = n >> 2;
+        constexpr int U = 8;
+        long long k = threadIdx.x;
+        for (; k + (long long)(U - 1) * kMeanThreads < n4; k += (long long)U * kMeanThreads) {
+            float4 x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) x[u] = __ldg(v4 + k + (long long)u * kMeanThreads);
+#pragma unroll
+            for (int u = 0; u < U; ++u) s += ((double)x[u].x + (double)x[u].y) + ((double)x[u].z + (double)x[u].w);
+        }
+        for (; k < n4; k += kMeanThreads) {
+            const float4 x = __ldg(v4 + k);
+            s += ((double)x.x + (double)x.y) + ((double)x.z + (double)x.w);
+        }
+        done = n4 << 2;
     }
-    if (threadIdx.x == 0) *out = n > 0 ? (float)(red[0] / (double)n) : 0.f;
+    for (long long k = done + threadIdx.x; k < n; k += kMeanThreads) s += (double)v[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        s = red[threadIdx.x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (threadIdx.x == 0) *out = n > 0 ? (float)(s / (double)n) : 0.f;
+    }
 }
 
 }  // namespace skl
