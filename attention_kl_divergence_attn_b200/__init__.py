@@ -9,6 +9,8 @@ is missing or the device is not an sm_100 GPU, calls raise.
 Functions keep the C names:
   streamkl_fwd(q_t, k_t, q_s, k_s, ...) -> (kl, lse_t, lse_s, loss_mean)
   streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, ...) -> (dq_s, dk_s, dq_t, dk_t)
+The autograd wrapper with temperature scaling is in ``.autograd``
+(``streamkl_loss``).
 """
 from __future__ import annotations
 
@@ -58,8 +60,13 @@ def lib():
             L.streamkl_bwd_dk.restype = _I
             L.streamkl_bwd_dq.argtypes = L.streamkl_bwd_dk.argtypes
             L.streamkl_bwd_dq.restype = _I
+            L.streamkl_bwd_dloss_device.argtypes = ([_VP] * 4 + shape + [_VP] * 3 + [_VP, _VP, _F] + [_VP] * 4
+                                                    + [_VP, ctypes.c_size_t, _VP])
+            L.streamkl_bwd_dloss_device.restype = _I
             L.streamkl_loss_mean.argtypes = [_VP, ctypes.c_longlong, _VP, _VP]
             L.streamkl_loss_mean.restype = _I
+            L.streamkl_loss_reduce.argtypes = [_VP, ctypes.c_longlong, ctypes.c_double, _VP, _VP]
+            L.streamkl_loss_reduce.restype = _I
             L.streamkl_fwd_noalloc.argtypes = ([_VP] * 4 + shape + [_VP] * 4 + [_VP, ctypes.POINTER(ctypes.c_uint)])
             L.streamkl_fwd_noalloc.restype = _I
             L.streamkl_workspace_size.argtypes = [_I] * 7
@@ -77,17 +84,38 @@ def lib():
 
 
 _workspaces: dict = {}
+_ws_sizes: dict = {}
+_STATUS_BYTES = 256
 
 
-def workspace(device=None) -> torch.Tensor:
-    """This device's workspace (status word), created and cleared on first use."""
+def workspace(device=None, nbytes=None) -> torch.Tensor:
+    """This device's workspace, created and cleared on first use.
+
+    Its first 256 bytes are the library's device status word.  ``nbytes``
+    (from ``workspace_size``) grows it for problems whose kernels split key
+    ranges; growing keeps the status word.  Calls through this module run on
+    the current stream, so they are ordered and may share it.
+    """
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    need = max(int(nbytes or 0), _STATUS_BYTES)
     ws = _workspaces.get(dev.index)
-    if ws is None:
-        n = lib().streamkl_workspace_size(0, 0, 0, 0, 0, 0, 0)
-        ws = torch.zeros(max(int(n), 16), dtype=torch.uint8, device=dev)
+    if ws is None or ws.numel() < need:
+        new = torch.zeros(need, dtype=torch.uint8, device=dev)
+        if ws is not None:
+            new[:_STATUS_BYTES].copy_(ws[:_STATUS_BYTES])
+        ws = new
         _workspaces[dev.index] = ws
     return ws
+
+
+def workspace_size(B, H, N_Q, N_K, d_t, d_s, causal) -> int:
+    """streamkl_workspace_size for this problem on the current device (cached)."""
+    key = (torch.cuda.current_device(), B, H, N_Q, N_K, d_t, d_s, int(bool(causal)))
+    n = _ws_sizes.get(key)
+    if n is None:
+        n = int(lib().streamkl_workspace_size(B, H, N_Q, N_K, d_t, d_s, int(bool(causal))))
+        _ws_sizes[key] = n
+    return n
 
 
 def _ptr(t):
@@ -133,7 +161,7 @@ def streamkl_fwd(q_t, k_t, q_s, k_s, scale_t=None, scale_s=None, causal=False, *
     else:
         kl, lse_t, lse_s = out[:3]
         loss = (out[3] if len(out) > 3 else torch.empty((), dtype=torch.float32, device=dev)) if loss_mean else None
-    ws = workspace(dev)
+    ws = workspace(dev, workspace_size(B, H, N_Q, N_K, d_t, d_s, causal))
     rc = lib().streamkl_fwd(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
                             scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
                             _ptr(loss), _ptr(ws), ws.numel(), _stream(stream))
@@ -143,11 +171,14 @@ def streamkl_fwd(q_t, k_t, q_s, k_s, scale_t=None, scale_s=None, causal=False, *
 
 
 def streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=None, causal=False, *,
-                 dkl=None, dloss=1.0, teacher_grads=False, out=None, stream=None):
+                 dkl=None, dloss=1.0, dloss_scale=None, teacher_grads=False, out=None, stream=None):
     """Gradients of sum_i g_i KL_i with g = dkl, or of dloss * mean(KL) if dkl is None.
 
-    Returns (dq_s, dk_s, dq_t, dk_t), fp32, the teacher pair None unless
-    teacher_grads.  ``out`` may supply the four buffers.
+    ``dloss`` is a number or a 0-d CUDA fp32 tensor; a tensor stays on the
+    device (streamkl_bwd_dloss_device) and then g = dloss_scale * dloss, with
+    dloss_scale defaulting to 1 / (B*H*N_Q).  Returns (dq_s, dk_s, dq_t,
+    dk_t), fp32, the teacher pair None unless teacher_grads.  ``out`` may
+    supply the four buffers.
     """
     B, H, N_Q, N_K, d_t, d_s = _check_inputs(q_t, k_t, q_s, k_s)
     scale_t = 1.0 / math.sqrt(d_t) if scale_t is None else float(scale_t)
@@ -163,7 +194,20 @@ def streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t=None, scale_s=Non
         dk_t = torch.empty(B, H, N_K, d_t, dtype=torch.float32, device=dev) if teacher_grads else None
     else:
         dq_s, dk_s, dq_t, dk_t = out
-    ws = workspace(dev)
+    ws = workspace(dev, workspace_size(B, H, N_Q, N_K, d_t, d_s, causal))
+    if isinstance(dloss, torch.Tensor):
+        if dloss.dtype != torch.float32 or dloss.numel() != 1 or dloss.device != dev:
+            raise ValueError("a tensor dloss must be a one-element fp32 tensor on the inputs' device")
+        scale = 1.0 / (B * H * N_Q) if dloss_scale is None else float(dloss_scale)
+        rc = lib().streamkl_bwd_dloss_device(
+            _ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s,
+            int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s), _ptr(dkl), _ptr(dloss), scale,
+            _ptr(dq_s), _ptr(dk_s), _ptr(dq_t), _ptr(dk_t), _ptr(ws), ws.numel(), _stream(stream))
+        if rc:
+            raise StreamKLError("streamkl_bwd_dloss_device", rc)
+        return dq_s, dk_s, dq_t, dk_t
+    if dloss_scale is not None:
+        raise ValueError("dloss_scale applies to a device-tensor dloss only")
     rc = lib().streamkl_bwd(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
                             scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
                             _ptr(dkl), float(dloss), _ptr(dq_s), _ptr(dk_s), _ptr(dq_t), _ptr(dk_t),
@@ -185,7 +229,7 @@ def _bwd_part(fn, which, q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s,
         g_t = torch.empty(B, H, n, d_t, dtype=torch.float32, device=dev) if teacher_grads else None
     else:
         g_s, g_t = out
-    ws = workspace(dev)
+    ws = workspace(dev, workspace_size(B, H, N_Q, N_K, d_t, d_s, causal))
     rc = getattr(lib(), fn)(_ptr(q_t), _ptr(k_t), _ptr(q_s), _ptr(k_s), B, H, N_Q, N_K, d_t, d_s,
                             scale_t, scale_s, int(bool(causal)), _ptr(kl), _ptr(lse_t), _ptr(lse_s),
                             _ptr(dkl), float(dloss), _ptr(g_s), _ptr(g_t), _ptr(ws), ws.numel(), _stream(stream))
@@ -216,6 +260,17 @@ def streamkl_loss_mean(kl, out=None, stream=None):
     rc = lib().streamkl_loss_mean(_ptr(kl), kl.numel(), _ptr(out), _stream(stream))
     if rc:
         raise StreamKLError("streamkl_loss_mean", rc)
+    return out
+
+
+def streamkl_loss_reduce(kl, factor, out=None, stream=None):
+    """factor * sum(kl) (fixed order, fp64 accumulation) as a 0-d device tensor."""
+    if kl.dtype != torch.float32 or not kl.is_cuda or not kl.is_contiguous():
+        raise TypeError("kl must be a contiguous CUDA fp32 tensor")
+    out = torch.empty((), dtype=torch.float32, device=kl.device) if out is None else out
+    rc = lib().streamkl_loss_reduce(_ptr(kl), kl.numel(), float(factor), _ptr(out), _stream(stream))
+    if rc:
+        raise StreamKLError("streamkl_loss_reduce", rc)
     return out
 
 

@@ -52,14 +52,22 @@ namespace skl {
 
 struct BwdParams {
     int BH, N_Q, N_K, causal, n_tiles;
+    int splits;                   // query-owner kernel: key ranges per query tile (1 = whole row)
     float ct, cs;                 // scale * log2(e)
     float out_t, out_s;           // output scales: scale_t * ln2 (teacher), scale_s (student)
     const float *kl, *lse_t, *lse_s, *dkl;
-    float g_const;                // g when dkl == nullptr
+    float g_const;                // g when dkl == nullptr (times *g_dev when g_dev != nullptr)
+    const float *g_dev;           // optional device scalar factor of g_const
     float inv_scale_t, inv_scale_s;
     float *dq_s, *dq_t, *dk_s, *dk_t;
+    float *part_s, *part_t;       // splits > 1: per-split dQ partials [splits][BH*N_Q][d]
     DevStatus st;
 };
+
+// The upstream gradient shared by all rows when no per-row dkl is given.
+__device__ __forceinline__ float uniform_g(const BwdParams &p) {
+    return p.g_dev ? p.g_const * __ldg(p.g_dev) : p.g_const;
+}
 
 constexpr float kLog2eF = 1.4426950408889634074f;
 
@@ -307,6 +315,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         // are fetched from global memory two tiles ahead into registers, with loads
         // the compiler may not move (ld_now), so that their latency overlaps the
         // tiles in between instead of stalling the ring.
+        const float g_all = uniform_g(p);
         auto load_consts = [&](int t, float4 (&v)[2]) {   // raw {lse_t, lse_s, g, kl}
             const int q0 = (first_qt + t) * C::BM;
 #pragma unroll
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     const size_t r = (size_t)bh * p.N_Q + i;
                     v[h].x = ld_now(p.lse_t + r);
                     v[h].y = ld_now(p.lse_s + r);
-                    v[h].z = p.dkl ? ld_now(p.dkl + r) : p.g_const;
+                    v[h].z = p.dkl ? ld_now(p.dkl + r) : g_all;
                     v[h].w = ld_now(p.kl + r);
                 }
             }
@@ -510,13 +519,19 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt_idx = p.n_tiles - 1 - (int)(blockIdx.x / p.BH);
+    // heaviest causal query tiles first; the key splits of a tile are adjacent
+    const int lin = (int)(blockIdx.x / p.BH);
+    const int split = lin % p.splits;
+    const int qt_idx = p.n_tiles - 1 - lin / p.splits;
     const int bh = (int)(blockIdx.x % p.BH);
     const int q0 = qt_idx * C::BM;
     const int off = p.N_K - p.N_Q;
     int kend = p.N_K;
     if (p.causal) kend = min(p.N_K, min(q0 + C::BM - 1, p.N_Q - 1) + off + 1);
-    const int n_kt = (kend + C::BN - 1) / C::BN;
+    const int n_all = (kend + C::BN - 1) / C::BN;
+    // this CTA's key tiles [kt_lo, kt_lo + n_kt) (the host keeps n_kt >= 1); loops count from 0
+    const int kt_lo = (int)((long long)n_all * split / p.splits);
+    const int n_kt = (int)((long long)n_all * (split + 1) / p.splits) - kt_lo;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar_q, 1);
@@ -559,10 +574,11 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bh);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
+                                bh);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -636,7 +652,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             const size_t r = (size_t)bh * p.N_Q + gq;
             Lt = p.lse_t[r] * kLog2eF;
             Ls = p.lse_s[r] * kLog2eF;
-            g = p.dkl ? p.dkl[r] : p.g_const;
+            g = p.dkl ? p.dkl[r] : uniform_g(p);
             KL2 = p.kl[r] * kLog2eF;
         }
         const int lim = p.causal ? min(p.N_K, gq + off + 1) : p.N_K;   // first hidden key
@@ -647,7 +663,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
 #pragma unroll
             for (int cc = 0; cc < C::CW / 32; ++cc) {
                 const int c = half * (C::CW / 32) + cc;   // chunk of the tile
-                const int kb = kt * C::BN + c * 32;
+                const int kb = (kt_lo + kt) * C::BN + c * 32;
                 const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
                 if (masked)
                     dq_chunk<TEACHER, true>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
@@ -662,10 +678,16 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();
             const bool store = gq < p.N_Q;
-            const size_t r = (size_t)bh * p.N_Q + (store ? gq : 0);
+            size_t r = (size_t)bh * p.N_Q + (store ? gq : 0);
+            float *dst_s = p.dq_s, *dst_t = p.dq_t;
+            if (p.splits > 1) {             // this split's partial, summed by streamkl_split_sum_kernel
+                r += (size_t)split * p.BH * p.N_Q;
+                dst_s = p.part_s;
+                dst_t = p.part_t;
+            }
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
-            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s, p.dq_s + r * DS + wg * HS, store);
-            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t, p.dq_t + r * DT + wg * HT, store);
+            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s, dst_s + r * DS + wg * HS, store);
+            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t, dst_t + r * DT + wg * HT, store);
         }
     }
 
@@ -674,6 +696,23 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// out[i] = sum over s of part[s * n + i], s in order (deterministic); n % 4 == 0
+// and 16-byte aligned arrays (gradient rows are 64 or 128 floats).
+__global__ void __launch_bounds__(256) streamkl_split_sum_kernel(const float *__restrict__ part, int splits,
+                                                                 long long n, float *__restrict__ out) {
+    const long long n4 = n >> 2;
+    const float4 *p4 = reinterpret_cast<const float4 *>(part);
+    float4 *o4 = reinterpret_cast<float4 *>(out);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        float4 a = __ldg(p4 + i);
+        for (int s = 1; s < splits; ++s) {
+            const float4 b = __ldg(p4 + (long long)s * n4 + i);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        o4[i] = a;
     }
 }
 

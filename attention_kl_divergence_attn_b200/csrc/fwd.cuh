@@ -36,10 +36,42 @@ namespace skl {
 
 struct FwdParams {
     int BH, N_Q, N_K, causal, n_qt;
+    int splits;            // key ranges per query tile (1 = the whole row in one CTA)
     float ct, cs;          // scale_t * log2(e), scale_s * log2(e)
     float *kl, *lse_t, *lse_s;
+    float *part;           // splits > 1: partial states, field f of split s, row r at [(f*splits + s)*rows + r]
     DevStatus st;
 };
+
+// Online state of one row over a set of keys (log2 units, see above).
+struct RowState {
+    float Mt, Ms, lt, ls, A;
+};
+
+// Folds state b into a: both rescaled to the larger maxima (teacher maximum
+// for l_t and A, student maximum for l_s).  Associative and exact up to
+// rounding; a state with no visible key (M = -inf, sums 0) is the identity.
+__device__ __forceinline__ void merge_state(RowState &a, const RowState &b) {
+    const float nMt = fmaxf(a.Mt, b.Mt), nMs = fmaxf(a.Ms, b.Ms);
+    if (nMt == -INFINITY) return;
+    const float a1 = ex2(a.Mt - nMt), a2 = ex2(b.Mt - nMt);
+    const float b1 = ex2(a.Ms - nMs), b2 = ex2(b.Ms - nMs);
+    a.lt = a.lt * a1 + b.lt * a2;
+    a.A = a.A * a1 + b.A * a2;
+    a.ls = a.ls * b1 + b.ls * b2;
+    a.Mt = nMt;
+    a.Ms = nMs;
+}
+
+// Row outputs from a complete state: LSE = ln2 (M + log2 l) for each
+// distribution and KL = ln2 (A / l_t) - LSE_t + LSE_s.
+__device__ __forceinline__ void finish_row(const RowState &x, float *kl, float *lse_t, float *lse_s) {
+    const float LN2 = 0.69314718055994530942f;
+    const float lse_t2 = x.Mt + lg2(x.lt), lse_s2 = x.Ms + lg2(x.ls);
+    *lse_t = lse_t2 * LN2;
+    *lse_s = lse_s2 * LN2;
+    *kl = LN2 * (x.A / x.lt - lse_t2 + lse_s2);
+}
 
 template <int DT, int DS, int NWG>
 struct FwdCfg {
@@ -171,11 +203,17 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // heaviest (latest) causal query tiles first
-    const int qt_idx = p.n_qt - 1 - (int)(blockIdx.x / p.BH);
+    // heaviest (latest) causal query tiles first; with key splits, the splits
+    // of one query tile are adjacent in launch order
+    const int lin = (int)(blockIdx.x / p.BH);
+    const int split = lin % p.splits;
+    const int qt_idx = p.n_qt - 1 - lin / p.splits;
     const int bh = (int)(blockIdx.x % p.BH);
     const int q0 = qt_idx * C::BM;
-    const int n_kt = fwd_key_tiles(q0, p.N_Q, p.N_K, p.causal, C::BN);
+    const int n_all = fwd_key_tiles(q0, p.N_Q, p.N_K, p.causal, C::BN);
+    // this CTA's key tiles [kt_lo, kt_lo + n_kt); loops below count from 0
+    const int kt_lo = (int)((long long)n_all * split / p.splits);
+    const int n_kt = (int)((long long)n_all * (split + 1) / p.splits) - kt_lo;
     const int off = p.N_K - p.N_Q;
 
     if (threadIdx.x == 0) {
@@ -218,10 +256,11 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bh);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, kt * C::BN, bh);
+                    tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
+                                bh);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -278,7 +317,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             const uint32_t bufc = lane_base + buf * 128;
             if (!mbar_wait(&bar_sfull[buf], (kt / C::NBUF) & 1, p.st, abort_v, 5)) break;
             tc_fence_after();
-            const int k0 = kt * C::BN;
+            const int k0 = (kt_lo + kt) * C::BN;
 #pragma unroll
             for (int cc = 0; cc < C::CW / 32; ++cc) {
                 const int c = half * (C::CW / 32) + cc;
@@ -303,6 +342,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_sempty[buf]);
         }
+        RowState x{Mt, Ms, lt, ls, A};
         if (NWG > 1) {
             if (wg > 0) {
                 merge[wg - 1][0][row] = Mt; merge[wg - 1][1][row] = Ms; merge[wg - 1][2][row] = lt;
@@ -311,28 +351,20 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             asm volatile("bar.sync 1, %0;" ::"r"(128 * NWG) : "memory");
             if (wg == 0) {
 #pragma unroll
-                for (int o = 0; o < NWG - 1; ++o) {
-                    const float Mt2 = merge[o][0][row], Ms2 = merge[o][1][row];
-                    const float nMt = fmaxf(Mt, Mt2), nMs = fmaxf(Ms, Ms2);
-                    if (nMt != -INFINITY) {
-                        const float a1 = ex2(Mt - nMt), a2 = ex2(Mt2 - nMt);
-                        const float b1 = ex2(Ms - nMs), b2 = ex2(Ms2 - nMs);
-                        lt = lt * a1 + merge[o][2][row] * a2;
-                        A = A * a1 + merge[o][4][row] * a2;
-                        ls = ls * b1 + merge[o][3][row] * b2;
-                        Mt = nMt;
-                        Ms = nMs;
-                    }
-                }
+                for (int o = 0; o < NWG - 1; ++o)
+                    merge_state(x, RowState{merge[o][0][row], merge[o][1][row], merge[o][2][row], merge[o][3][row],
+                                            merge[o][4][row]});
             }
         }
         if (wg == 0 && grow < p.N_Q && !*abort_v) {
-            const float LN2 = 0.69314718055994530942f;
-            const float lse_t2 = Mt + lg2(lt), lse_s2 = Ms + lg2(ls);
             const size_t r = (size_t)bh * p.N_Q + grow;
-            p.lse_t[r] = lse_t2 * LN2;
-            p.lse_s[r] = lse_s2 * LN2;
-            p.kl[r] = LN2 * (A / lt - lse_t2 + lse_s2);
+            if (p.splits > 1) {
+                const size_t rows = (size_t)p.BH * p.N_Q, fs = (size_t)p.splits * rows;
+                float *q = p.part + (size_t)split * rows + r;
+                q[0] = x.Mt; q[fs] = x.Ms; q[2 * fs] = x.lt; q[3 * fs] = x.ls; q[4 * fs] = x.A;
+            } else {
+                finish_row(x, p.kl + r, p.lse_t + r, p.lse_s + r);
+            }
         }
     }
 
@@ -344,14 +376,33 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     }
 }
 
-// Deterministic mean of n per-row values: one CTA of kMeanThreads threads,
-// each summing a fixed strided subset in fp64 (16-byte loads, eight in flight
-// per thread when the array is 16-byte aligned), then a fixed-shape tree
-// (warp shuffles, then one warp over the warp sums).  The order of additions
-// depends only on n, so the result is the same run to run.
+// Combines the partial states of the key splits of every row, in split
+// order (so the result is the same run to run), and writes the row outputs.
+__global__ void __launch_bounds__(256) streamkl_fwd_merge_kernel(const float *__restrict__ part, int splits,
+                                                                 long long rows, float *__restrict__ kl,
+                                                                 float *__restrict__ lse_t,
+                                                                 float *__restrict__ lse_s) {
+    const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const long long fs = (long long)splits * rows;
+    RowState x{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+    for (int s = 0; s < splits; ++s) {
+        const float *q = part + (long long)s * rows + r;
+        merge_state(x, RowState{q[0], q[fs], q[2 * fs], q[3 * fs], q[4 * fs]});
+    }
+    finish_row(x, kl + r, lse_t + r, lse_s + r);
+}
+
+// Deterministic reduction of n per-row values: out = (sum / div) * mul (the
+// mean with div = n, mul = 1).  One CTA of kMeanThreads threads, each summing
+// a fixed strided subset in fp64 (16-byte loads, eight in flight per thread
+// when the array is 16-byte aligned), then a fixed-shape tree (warp shuffles,
+// then one warp over the warp sums).  The order of additions depends only on
+// n, so the result is the same run to run.
 constexpr int kMeanThreads = 1024;
 
 __global__ void __launch_bounds__(kMeanThreads) streamkl_mean_kernel(const float *__restrict__ v, long long n,
+                                                                     double div, double mul,
                                                                      float *__restrict__ out) {
     __shared__ double red[kMeanThreads / 32];
     double s = 0.0;
@@ -383,7 +434,7 @@ __global__ void __launch_bounds__(kMeanThreads) streamkl_mean_kernel(const float
         s = red[threadIdx.x];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (threadIdx.x == 0) *out = n > 0 ? (float)(s / (double)n) : 0.f;
+        if (threadIdx.x == 0) *out = n > 0 ? (float)((s / div) * mul) : 0.f;
     }
 }
 

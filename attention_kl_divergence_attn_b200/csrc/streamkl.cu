@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include <cuda.h>
@@ -84,15 +85,65 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 constexpr int kFwdWarpgroups = 4;
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+// Key splits for the kernels that own 128-row query tiles and walk 64-key
+// tiles (the forward and the query-owner backward).  With few query tiles
+// (short N_Q, long N_K) one CTA per tile leaves SMs idle in the last wave, so
+// each tile's key range is cut into S pieces that run as separate CTAs and
+// are combined afterwards (forward: the associative merge of the online
+// states; backward: a fixed-order sum of dQ partials).  S minimises
+// waves(S) / S, the estimated time in units of one whole-row CTA, with 2 %
+// added per extra piece for the combine pass and per-CTA set-up; every piece
+// keeps at least kMinSplitTiles key tiles of the shortest (first, under
+// causal) query tile.
+constexpr int kMaxSplits = 32, kMinSplitTiles = 4;
+
+int key_splits(int BH, int N_Q, int N_K, int causal) {
+    const int sms = sm_count();
+    const long long ctas = (long long)BH * ((N_Q + 127) / 128);
+    if (sms <= 0 || ctas == 0 || ctas >= 8ll * sms) return 1;
+    int kend = N_K;
+    if (causal) kend = std::min(N_K, std::min(127, N_Q - 1) + (N_K - N_Q) + 1);
+    const int smax = std::min(kMaxSplits, ((kend + 63) / 64) / kMinSplitTiles);
+    int best = 1;
+    double best_t = 1e300;
+    for (int S = 1; S <= std::max(1, smax); ++S) {
+        const double waves = (double)((ctas * S + sms - 1) / sms);
+        const double t = waves / S * (1.0 + 0.02 * (S - 1));
+        if (t < best_t * (1.0 - 1e-9)) { best = S; best_t = t; }
+    }
+    return best;
+}
+
+// Workspace bytes beyond the status word that S key splits need.
+size_t fwd_split_bytes(int S, long long rows) { return S > 1 ? (size_t)5 * S * rows * sizeof(float) : 0; }
+size_t dq_split_bytes(int S, long long rows, int d_s, int d_t) {
+    return S > 1 ? (size_t)S * rows * (d_s + d_t) * sizeof(float) : 0;
+}
+
 template <int DT, int DS>
 streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const CUtensorMap &qs,
                            const CUtensorMap &ks, const FwdParams &p, cudaStream_t stream) {
     using C = FwdCfg<DT, DS, kFwdWarpgroups>;
     auto kern = streamkl_fwd_kernel<DT, DS, kFwdWarpgroups>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
-    const long long grid = (long long)p.BH * p.n_qt;
+    const long long grid = (long long)p.BH * p.n_qt * p.splits;
     kern<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
-    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    if (p.splits > 1) {
+        const long long rows = (long long)p.BH * p.N_Q;
+        streamkl_fwd_merge_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(p.part, p.splits, rows, p.kl,
+                                                                                      p.lse_t, p.lse_s);
+        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    return STREAMKL_OK;
 }
 
 // Which backward kernels a call launches.
@@ -124,8 +175,20 @@ streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, co
         auto kdq = streamkl_bwd_dq_kernel<DT, DS, TEACHER>;
         if (set_smem(kdq, CQ::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
         p.n_tiles = (N_Q + CQ::BM - 1) / CQ::BM;
-        kdq<<<(unsigned)((long long)BH * p.n_tiles), CQ::THREADS, CQ::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        kdq<<<(unsigned)((long long)BH * p.n_tiles * p.splits), CQ::THREADS, CQ::SMEM, stream>>>(mqt, mkt, mqs,
+                                                                                              mks, p);
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+        if (p.splits > 1) {
+            const long long rows = (long long)BH * N_Q;
+            const int sms = std::max(1, sm_count());
+            for (int side = 0; side < (TEACHER ? 2 : 1); ++side) {
+                const long long n = rows * (side ? DT : DS);
+                const long long blocks = std::min<long long>((n / 4 + 255) / 256, 8ll * sms);
+                streamkl_split_sum_kernel<<<(unsigned)blocks, 256, 0, stream>>>(side ? p.part_t : p.part_s, p.splits,
+                                                                                 n, side ? p.dq_t : p.dq_s);
+                if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+            }
+        }
     }
     return STREAMKL_OK;
 }
@@ -144,8 +207,8 @@ streamkl_status dispatch_bwd(int d_t, int d_s, const void *q_t, const void *k_t,
 streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
                            int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
                            const float *kl, const float *lse_t, const float *lse_s, const float *dkl, float dloss,
-                           float *dq_s, float *dk_s, float *dq_t, float *dk_t, void *workspace,
-                           size_t workspace_bytes, void *stream, int parts) {
+                           const float *dloss_dev, float *dq_s, float *dk_s, float *dq_t, float *dk_t,
+                           void *workspace, size_t workspace_bytes, void *stream, int parts) {
     streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
     if (st != STREAMKL_OK) return st;
     if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
@@ -182,12 +245,27 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     p.out_t = scale_t * 0.69314718055994530942f;
     p.out_s = scale_s;
     p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s; p.dkl = dkl;
-    p.g_const = (float)((double)dloss / ((double)BH * (double)N_Q));
+    if (dloss_dev) {                 // g = dloss (a scale) times the device scalar
+        p.g_const = dloss;
+        p.g_dev = dloss_dev;
+    } else {
+        p.g_const = (float)((double)dloss / ((double)BH * (double)N_Q));
+    }
     p.inv_scale_t = 1.0f / scale_t;
     p.inv_scale_s = 1.0f / scale_s;
     p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
     p.st.word = static_cast<uint32_t *>(workspace);
     p.st.budget_ns = kWaitBudgetNs;
+    p.splits = 1;
+    if (want_dq) {
+        const long long rows = (long long)BH * N_Q;
+        const int S = key_splits(BH, N_Q, N_K, causal);
+        if (S > 1 && workspace_bytes >= kWorkspaceBytes + dq_split_bytes(S, rows, d_s, teacher ? d_t : 0)) {
+            p.splits = S;
+            p.part_s = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWorkspaceBytes);
+            p.part_t = p.part_s + (size_t)S * rows * d_s;
+        }
+    }
     return teacher ? dispatch_bwd<true>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s)
                    : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
 }
@@ -198,7 +276,14 @@ extern "C" {
 
 int streamkl_version(void) { return 100; }
 
-size_t streamkl_workspace_size(int, int, int, int, int, int, int) { return kWorkspaceBytes; }
+size_t streamkl_workspace_size(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal) {
+    if (B <= 0 || H <= 0 || N_Q <= 0 || N_K <= 0 || (d_t != 64 && d_t != 128) || (d_s != 64 && d_s != 128))
+        return kWorkspaceBytes;
+    const long long rows = (long long)B * H * N_Q;
+    const int S = key_splits(B * H, N_Q, N_K, causal ? 1 : 0);
+    const size_t extra = std::max(fwd_split_bytes(S, rows), dq_split_bytes(S, rows, d_s, d_t));
+    return kWorkspaceBytes + ((extra + 255) / 256) * 256;
+}
 
 const char *streamkl_strerror(streamkl_status s) {
     switch (s) {
@@ -247,7 +332,7 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     const int BH = B * H;
     const long long rows = (long long)BH * N_Q;
     if (rows == 0) {
-        if (loss_mean) streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, 0, loss_mean);
+        if (loss_mean) streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
         return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
     }
     if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
@@ -266,13 +351,22 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s;
     p.st.word = static_cast<uint32_t *>(workspace);
     p.st.budget_ns = kWaitBudgetNs;
+    p.splits = 1;
+    p.part = nullptr;
+    {
+        const int S = key_splits(BH, N_Q, N_K, causal);
+        if (S > 1 && workspace_bytes >= kWorkspaceBytes + fwd_split_bytes(S, rows)) {
+            p.splits = S;
+            p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWorkspaceBytes);
+        }
+    }
     if (d_t == 64 && d_s == 64) st = launch_fwd<64, 64>(mqt, mkt, mqs, mks, p, s);
     else if (d_t == 128 && d_s == 128) st = launch_fwd<128, 128>(mqt, mkt, mqs, mks, p, s);
     else if (d_t == 128 && d_s == 64) st = launch_fwd<128, 64>(mqt, mkt, mqs, mks, p, s);
     else st = launch_fwd<64, 128>(mqt, mkt, mqs, mks, p, s);
     if (st != STREAMKL_OK) return st;
     if (loss_mean) {
-        streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, rows, loss_mean);
+        streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, rows, (double)rows, 1.0, loss_mean);
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
     }
     return STREAMKL_OK;
@@ -286,7 +380,7 @@ streamkl_status streamkl_bwd(const void *q_t, const void *k_t, const void *q_s, 
                              float *dq_s, float *dk_s, float *dq_t, float *dk_t, void *workspace,
                              size_t workspace_bytes, void *stream) {
     return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
-                      dloss, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes, stream, kPartDK | kPartDQ);
+                      dloss, nullptr, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes, stream, kPartDK | kPartDQ);
 }
 
 streamkl_status streamkl_bwd_dk(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
@@ -295,7 +389,7 @@ streamkl_status streamkl_bwd_dk(const void *q_t, const void *k_t, const void *q_
                                 float dloss, float *dk_s, float *dk_t, void *workspace, size_t workspace_bytes,
                                 void *stream) {
     return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
-                      dloss, nullptr, dk_s, nullptr, dk_t, workspace, workspace_bytes, stream, kPartDK);
+                      dloss, nullptr, nullptr, dk_s, nullptr, dk_t, workspace, workspace_bytes, stream, kPartDK);
 }
 
 streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
@@ -304,12 +398,30 @@ streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_
                                 float dloss, float *dq_s, float *dq_t, void *workspace, size_t workspace_bytes,
                                 void *stream) {
     return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
-                      dloss, dq_s, nullptr, dq_t, nullptr, workspace, workspace_bytes, stream, kPartDQ);
+                      dloss, nullptr, dq_s, nullptr, dq_t, nullptr, workspace, workspace_bytes, stream, kPartDQ);
+}
+
+streamkl_status streamkl_bwd_dloss_device(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B,
+                                          int H, int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s,
+                                          int causal, const float *kl, const float *lse_t, const float *lse_s,
+                                          const float *dkl, const float *dloss_dev, float dloss_scale, float *dq_s,
+                                          float *dk_s, float *dq_t, float *dk_t, void *workspace,
+                                          size_t workspace_bytes, void *stream) {
+    if (!dkl && !dloss_dev) return STREAMKL_ERR_INVALID_ARG;
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+                      dloss_scale, dkl ? nullptr : dloss_dev, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes,
+                      stream, kPartDK | kPartDQ);
 }
 
 streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream) {
     if (n_rows < 0 || !loss_mean || (n_rows > 0 && !kl)) return STREAMKL_ERR_INVALID_ARG;
-    streamkl_mean_kernel<<<1, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, loss_mean);
+    streamkl_mean_kernel<<<1, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, (double)n_rows, 1.0, loss_mean);
+    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+}
+
+streamkl_status streamkl_loss_reduce(const float *kl, long long n_rows, double factor, float *out, void *stream) {
+    if (n_rows < 0 || !out || (n_rows > 0 && !kl) || !(factor == factor)) return STREAMKL_ERR_INVALID_ARG;
+    streamkl_mean_kernel<<<1, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, 1.0, factor, out);
     return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
@@ -356,8 +468,9 @@ extern "C" streamkl_status streamkl_fwd_noalloc(const void *q_t, const void *k_t
                                                 int B, int H, int N_Q, int N_K, int d_t, int d_s, float scale_t,
                                                 float scale_s, int causal, float *kl, float *lse_t, float *lse_s,
                                                 float *loss_mean, void *stream, unsigned int *status_out) {
-    if (streamkl_workspace_size(B, H, N_Q, N_K, d_t, d_s, causal) > kNoAllocScratchBytes)
-        return STREAMKL_ERR_WORKSPACE;          // this problem needs more scratch than the array holds
+    // every problem runs with the minimum workspace (key splitting, which
+    // needs more, is only used when the caller's workspace has room for it)
+    static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "the array holds the minimum workspace");
     void *scratch = nullptr;
     streamkl_status st = noalloc_scratch(&scratch);
     if (st != STREAMKL_OK) return st;

@@ -32,11 +32,19 @@
  *    stream) and is asynchronous: a return of STREAMKL_OK means the launch was
  *    accepted.  Errors found on the device (a bounded wait that gave up) are
  *    recorded in the caller's workspace and reported by streamkl_check().
- *  - `workspace` is device memory of at least streamkl_workspace_size() bytes,
- *    owned by the caller, cleared once with streamkl_workspace_init() before
- *    first use.  It holds a sticky device status word that kernels set when a
- *    bounded wait gives up; streamkl_check() reads and clears it.  Calls that
- *    share one workspace may overlap on the GPU (the word is only OR-ed).
+ *  - `workspace` is device memory owned by the caller, at least 256 bytes,
+ *    cleared once with streamkl_workspace_init() before first use.  Its first
+ *    256 bytes hold a sticky device status word that kernels set when a
+ *    bounded wait gives up; streamkl_check() reads and clears it.  A
+ *    workspace of streamkl_workspace_size() bytes (more than 256 only for
+ *    problems with few query tiles and long key ranges) also lets the
+ *    forward and the query-side backward split each query tile's keys across
+ *    several CTAs (partial results go to the bytes after the status word and
+ *    are combined in a fixed order, so results are the same run to run;
+ *    they match the unsplit path up to rounding).  Calls that share a
+ *    256-byte workspace may overlap on the GPU (the word is only OR-ed);
+ *    calls that share a larger one must be ordered (one stream), since their
+ *    partial results would collide.
  *  - No entry point aborts, prints, or allocates; on an argument error nothing
  *    is launched.
  */
@@ -58,8 +66,14 @@ typedef enum {
     STREAMKL_ERR_WORKSPACE = 5      /* workspace NULL or smaller than streamkl_workspace_size() */
 } streamkl_status;
 
-/* Bytes of device workspace a call needs for this problem (a small constant:
- * the device status word; nothing grows with N_Q or N_K). */
+/* Bytes of device workspace that let streamkl_fwd and streamkl_bwd run this
+ * problem on their fastest path on the current device: 256 (the status word)
+ * plus, when the problem has too few 128-row query tiles to fill the GPU and
+ * long enough key ranges, room for the partial results of key splits
+ * (5 floats per row and split for the forward, d_s + d_t floats per row and
+ * split for the query-side backward; at most a few tens of MB).  Any
+ * workspace of at least 256 bytes is accepted; a smaller one than this
+ * value only turns splitting off.  Arguments as in streamkl_fwd. */
 size_t streamkl_workspace_size(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal);
 
 /*
@@ -122,10 +136,35 @@ streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_
                                 const float *dkl, float dloss, float *dq_s, float *dq_t,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * streamkl_bwd with the scalar upstream gradient in DEVICE memory, so that a
+ * caller such as an autograd engine never reads it back to the host:
+ *   g_i = dkl[i]                       if dkl != NULL
+ *   g_i = dloss_scale * (*dloss_dev)   otherwise (dloss_dev: device fp32 scalar)
+ * e.g. dloss_scale = 1 / (B*H*N_Q) for the gradient of the mean loss, or
+ * T^2 / (B*H*N_Q) for the temperature-scaled distillation loss
+ * T^2 * mean KL ("Lecture 05 - Where It All Lands ...", section 3.3).
+ * Every other argument, result and error as streamkl_bwd; both dkl and
+ * dloss_dev NULL is STREAMKL_ERR_INVALID_ARG.
+ */
+streamkl_status streamkl_bwd_dloss_device(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                          int B, int H, int N_Q, int N_K, int d_t, int d_s,
+                                          float scale_t, float scale_s, int causal,
+                                          const float *kl, const float *lse_t, const float *lse_s,
+                                          const float *dkl, const float *dloss_dev, float dloss_scale,
+                                          float *dq_s, float *dk_s, float *dq_t, float *dk_t,
+                                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* loss_mean (device scalar) = mean of kl[0..n_rows) in a fixed summation
  * order (so repeated calls give identical bits); the same reduction
  * streamkl_fwd runs when its loss_mean argument is non-NULL. */
 streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream);
+
+/* out (device scalar) = factor * sum of kl[0..n_rows), same fixed order and
+ * fp64 accumulation as streamkl_loss_mean; factor = T^2 gives the summed
+ * temperature-scaled loss, T^2 / n_rows its mean.  A NaN factor is
+ * STREAMKL_ERR_INVALID_ARG. */
+streamkl_status streamkl_loss_reduce(const float *kl, long long n_rows, double factor, float *out, void *stream);
 
 /* Clears the workspace (enqueued on `stream`).  Needed once per workspace. */
 streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
@@ -154,8 +193,10 @@ streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int
  *  - Each call clears the status word at its start.  All calls on a device
  *    share the one array and it keeps the last call's contents, so calls that
  *    overlap on the GPU (different streams, no ordering) race on it.
- *  - A problem whose scratch need (streamkl_workspace_size) exceeds the array
- *    is rejected with STREAMKL_ERR_WORKSPACE before anything is launched.
+ *  - The array holds the 256-byte minimum workspace that every problem runs
+ *    with; the forward then does not split key ranges across CTAs (that
+ *    needs the larger workspace streamkl_workspace_size reports), so no
+ *    problem is rejected for size.
  *  - status_out (host pointer): if non-NULL the call synchronises `stream`,
  *    stores the device status word there (0 = clean) and returns
  *    STREAMKL_ERR_TIMEOUT if a bounded wait gave up; if NULL the call returns

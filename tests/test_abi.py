@@ -82,3 +82,24 @@ def test_misaligned_pointer_rejected(L):
     bad = ctypes.c_void_p(18)
     rc = L.streamkl_fwd(bad, p, p, p, 1, 1, 128, 128, 64, 64, 0.125, 0.125, 0, p, p, p, None, p, 256, None)
     assert rc == 1
+
+
+def test_device_scalar_backward_needs_a_gradient(L):
+    p = ctypes.c_void_p(16)
+    rc = L.streamkl_bwd_dloss_device(p, p, p, p, 1, 1, 128, 128, 64, 64, 0.125, 0.125, 0, p, p, p, None, None, 1.0,
+                                     p, p, None, None, ctypes.c_void_p(16), 256, None)
+    assert rc == 1
+
+
+def test_loss_reduce_argument_errors(L):
+    p = ctypes.c_void_p(16)
+    assert L.streamkl_loss_reduce(p, 10, float("nan"), p, None) == 1
+    assert L.streamkl_loss_reduce(p, -1, 1.0, p, None) == 1
+    assert L.streamkl_loss_reduce(p, 10, 1.0, None, None) == 1
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device answer")
+def test_workspace_size_minimum_without_gpu(L):
+    # no device: no key splitting is planned, so the minimum is reported
+    assert L.streamkl_workspace_size(4, 8, 1024, 65536, 128, 64, 0) == 256
+    assert L.streamkl_workspace_size(0, 0, 0, 0, 0, 0, 0) == 256
