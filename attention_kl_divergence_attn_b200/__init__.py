@@ -75,6 +75,8 @@ def lib():
             L.streamkl_workspace_init.restype = _I
             L.streamkl_check.argtypes = [_VP, _VP, ctypes.POINTER(ctypes.c_uint)]
             L.streamkl_check.restype = _I
+            L.streamkl_selftest_timeout.argtypes = [_VP, ctypes.c_size_t, ctypes.c_ulonglong, _VP]
+            L.streamkl_selftest_timeout.restype = _I
             L.streamkl_strerror.argtypes = [_I]
             L.streamkl_strerror.restype = ctypes.c_char_p
             L.streamkl_version.argtypes = []

@@ -270,9 +270,43 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
                    : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
 }
 
+// Self-test of the failure path: one warp waits, with the library's bounded
+// wait, on an mbarrier that nothing ever arrives at.  After `budget_ns` the
+// wait records a timeout (who = kSelftestWho) in the status word, raises the
+// CTA's abort flag (the other threads see it and return too) and the kernel
+// ends normally, so the caller can check that the timeout is reported and that
+// the CUDA context is still usable.  Nothing faults or hangs.
+constexpr uint32_t kSelftestWho = 63;
+
+__global__ void streamkl_selftest_timeout_kernel(DevStatus st) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    mbar_wait(&bar, 0, st, &abort_flag, kSelftestWho);
+}
+
 }  // namespace
 
 extern "C" {
+
+streamkl_status streamkl_selftest_timeout(void *workspace, size_t workspace_bytes, unsigned long long budget_ns,
+                                          void *stream) {
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
+    if (budget_ns < 1000000ull || budget_ns > kWaitBudgetNs) return STREAMKL_ERR_INVALID_ARG;
+    streamkl_status st = check_device();
+    if (st != STREAMKL_OK) return st;
+    DevStatus ds;
+    ds.word = static_cast<uint32_t *>(workspace);
+    ds.budget_ns = budget_ns;
+    streamkl_selftest_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(ds);
+    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+}
 
 int streamkl_version(void) { return 100; }
 

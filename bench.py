@@ -13,6 +13,9 @@ per head, halved for causal masks (2.199 TFLOP per step here).
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
   python bench.py --impl reference ...    # the fp64 CPU oracle on the same workload
+  python bench.py --impl materialised ... # torch eager on the GPU, both N_Q x N_K
+                                          # distributions materialised (the
+                                          # baseline the fused method replaces)
 
 With N > 1 (torchrun, one process per GPU) every rank solves its own
 independent problem of the default size (heads are independent: no data-path
@@ -244,6 +247,69 @@ def run_reference(args, w):
     return 0
 
 
+# ----------------------------------------------------------------------------- materialised comparison
+
+def run_materialised(args, w):
+    """The computation the fused method replaces, in torch eager on one GPU:
+    both logit matrices and both log-softmax distributions are materialised
+    ([B, H, N_Q, N_K] fp32), the per-row KL is reduced from them and autograd
+    produces the same gradients.  Same FLOP count, so the value compares
+    directly; the peak device memory is reported next to it.  Rank 0 only."""
+    import torch
+    import torch.nn.functional as F
+    from attention_kl_divergence_attn_b200 import inputs
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = {"impl": "materialised", "metric": METRIC, "unit": "TFLOP/s", "n_gpus": 1,
+            "config": workload_config(w), "data": "synthetic", "dtype": "bf16 matmul, fp32 softmax/KL"}
+    try:
+        x = [t.to(dev) for t in inputs.make_inputs(w)]
+        for i, t in enumerate(x):
+            t.requires_grad_(i >= 2 or w.teacher_grads)
+        mask = None
+        if w.causal:
+            i = torch.arange(w.N_Q, device=dev)[:, None]
+            j = torch.arange(w.N_K, device=dev)[None, :]
+            mask = j > i + (w.N_K - w.N_Q)
+
+        def step():
+            for t in x:
+                t.grad = None
+            st = torch.matmul(x[0], x[1].transpose(-1, -2)).float() * w.scale_t
+            ss = torch.matmul(x[2], x[3].transpose(-1, -2)).float() * w.scale_s
+            if mask is not None:                  # finite fill: P = 0 there, and no inf - inf
+                st = st.masked_fill(mask, -1e9)
+                ss = ss.masked_fill(mask, -1e9)
+            logp, logq = F.log_softmax(st, -1), F.log_softmax(ss, -1)
+            kl = F.kl_div(logq, logp, reduction="none", log_target=True).sum(-1)
+            loss = kl.mean()
+            loss.backward()
+            return loss
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        steps = min(args.steps, 20)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            step()
+        t1.record()
+        torch.cuda.synchronize(dev)
+        ms = t0.elapsed_time(t1) / steps
+    except torch.cuda.OutOfMemoryError as exc:
+        print(json.dumps(dict(base, unavailable=f"out of device memory: {str(exc).splitlines()[0]}")), flush=True)
+        return 0
+    line = dict(base, value=step_flops(w) / (ms * 1e-3) / 1e12, ms_per_step=ms, steps=steps,
+                warmup=args.warmup, higher_is_better=True,
+                peak_device_bytes=int(torch.cuda.max_memory_allocated(dev)))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_config(w) -> dict:
     in_bytes = 2 * w.B * w.H * (w.N_Q * (w.d_t + w.d_s) + w.N_K * (w.d_t + w.d_s))
     return {"workload": w.name, "B": w.B, "H": w.H, "N_Q": w.N_Q, "N_K": w.N_K, "d_t": w.d_t, "d_s": w.d_s,
@@ -260,7 +326,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--impl", choices=["mine", "reference", "materialised"], default="mine")
     ap.add_argument("--workload", default="causal_8k_d128")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -270,6 +336,8 @@ def main():
     w = inputs.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.impl == "materialised":
+        return run_materialised(args, w)
 
     import torch
     import torch.distributed as dist
@@ -328,6 +396,20 @@ def main():
         step()
     torch.cuda.synchronize(dev)
     skl.streamkl_check(stream)
+
+    # memory proof: one step allocates nothing beyond the buffers above
+    torch.cuda.reset_peak_memory_stats(dev)
+    alloc0 = torch.cuda.memory_allocated(dev)
+    free0 = torch.cuda.mem_get_info(dev)[0]
+    step()
+    torch.cuda.synchronize(dev)
+    memory = {"extra_bytes_during_step": int(torch.cuda.max_memory_allocated(dev) - alloc0),
+              "device_free_delta_bytes": int(free0 - torch.cuda.mem_get_info(dev)[0]),
+              "workspace_bytes": int(skl.workspace(dev).numel()),
+              "materialised_fp32_bytes_per_distribution": B * H * NQ * NK * 4}
+    # launches per step: the four kernels, plus the combine kernels when key splits are planned
+    split = skl.workspace_size(B, H, NQ, NK, dt_, ds_, w.causal) > 256
+    launches_per_step = 4 + ((2 + (1 if w.teacher_grads else 0)) if split else 0)
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
@@ -416,7 +498,8 @@ def main():
                         for n in names},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
-            "gpu_launches": 4 * K,
+            "gpu_launches": launches_per_step * K,
+            "memory": memory,
             "clocks": sampler.summary(),
             "device_status": code,
         }

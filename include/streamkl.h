@@ -208,6 +208,19 @@ streamkl_status streamkl_fwd_noalloc(const void *q_t, const void *k_t, const voi
                                      float *kl, float *lse_t, float *lse_s, float *loss_mean,
                                      void *stream, unsigned int *status_out);
 
+/*
+ * Self-test of device failure reporting.  Launches one warp that waits, with
+ * the same bounded wait every kernel of the library uses, on a barrier that is
+ * never signalled; after budget_ns (1 ms .. 2 s, else STREAMKL_ERR_INVALID_ARG)
+ * the wait gives up, ORs STREAMKL's timeout bit and the waiter id 63 (bits
+ * 8..15) into the workspace status word, and the kernel returns normally.  A
+ * following streamkl_check() on the same workspace then returns
+ * STREAMKL_ERR_TIMEOUT and clears the word; the CUDA context stays usable.
+ * Nothing faults and nothing hangs.  For tests of callers' error handling.
+ */
+streamkl_status streamkl_selftest_timeout(void *workspace, size_t workspace_bytes, unsigned long long budget_ns,
+                                          void *stream);
+
 /* Static, human-readable name of a status. */
 const char *streamkl_strerror(streamkl_status status);
 

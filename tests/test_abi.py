@@ -103,3 +103,9 @@ def test_workspace_size_minimum_without_gpu(L):
     # no device: no key splitting is planned, so the minimum is reported
     assert L.streamkl_workspace_size(4, 8, 1024, 65536, 128, 64, 0) == 256
     assert L.streamkl_workspace_size(0, 0, 0, 0, 0, 0, 0) == 256
+
+
+def test_selftest_argument_errors(L):
+    assert L.streamkl_selftest_timeout(None, 256, 10000000, None) == 5
+    assert L.streamkl_selftest_timeout(ctypes.c_void_p(16), 256, 10, None) == 1            # budget too short
+    assert L.streamkl_selftest_timeout(ctypes.c_void_p(16), 256, 10 ** 10, None) == 1      # above 2 s
