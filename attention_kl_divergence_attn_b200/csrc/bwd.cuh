@@ -23,7 +23,8 @@
 //       are (1, 1, 1, 0, ...), B = the tile's rows (h, m, l, 0, ...) with
 //       h + m + l = -LSE / scale split into three bf16 terms (about fp32
 //       precision), so the accumulator holds q.k - LSE / scale directly.
-//       Only g and KL per query come from a small shared-memory table.
+//       Only KL per query (and g, when it varies per row) comes from a small
+//       shared-memory table, read with one broadcast load per pair of queries.
 //   streamkl_bwd_dq_kernel   CTA = 128 queries of one head; loops over 64-key
 //       tiles: S = Q K^T, dS, dQ += dS K.  Thread = query row; per-row
 //       constants live in registers.
@@ -32,16 +33,17 @@
 // for the side it does not own (measured at ~5.8 TB/s of L2 reductions on
 // B200, that traffic would cost more than the recompute).
 //
-// Pipeline (both kernels).  Gradient warpgroups ping-pong over tiles: tile t
-// goes to TMEM buffer t & 1 (S_t in columns [0,64), S_s in [64,128) of the
-// buffer) and to the warpgroups of parity t & 1; with NH = 2 halves per parity
-// each of those warpgroups takes 32 of the tile's 64 columns.  A warpgroup
-// reads its S columns in 32-column chunks and writes the chunk's bf16 dS
-// (16 packed columns) over the first half of the same chunk, which only it
-// reads; the MMA warp then uses those columns directly as the A operand of
-// the gradient MMA (tcgen05.mma with A in tensor memory), so dS never touches
-// shared memory.  Because MMAs issued by one thread execute in order, S of
-// tile t+2 can be issued into buffer t & 1 right after the gradient MMA of t.
+// Pipeline (both kernels).  Tile t goes to TMEM buffer t & 1 (S_t in columns
+// [0,64), S_s in [64,128) of the buffer); all four gradient warpgroups work on
+// every tile, each on its own 16-column chunk, so sixteen warps share the
+// exponentials of a tile while the MMA warp computes the logits of the next
+// tile in the other buffer.  A warpgroup reads its chunk in 8-column pieces
+// and writes the chunk's bf16 dS (8 packed columns) over the first half of
+// the same chunk, which only it reads; the MMA warp then uses those columns
+// directly as the A operand of the gradient MMA (tcgen05.mma with A in tensor
+// memory), so dS never touches shared memory.  Because MMAs issued by one
+// thread execute in order, S of tile t+2 can be issued into buffer t & 1 right
+// after the gradient MMA of t.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -102,22 +104,22 @@ __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float u
     if (TEACHER) pt = pack_bf16((g0 * P0) * ((at0 - as0) - K0), (g1 * P1) * ((at1 - as1) - K1));
 }
 
-// The two chunk routines below turn one 32-column chunk of a warpgroup's S
-// columns (teacher logits at `at`, student at `as`) into this thread's 32 dS
-// values, written as 16 packed bf16 columns over the first half of the chunk
-// (student dS over the teacher logits, teacher dS over the student logits).
+// The two chunk routines below turn one CWID-column chunk of a warpgroup's S
+// columns (teacher logits at `at`, student at `as`) into this thread's CWID dS
+// values, written as CWID/2 packed bf16 columns over the first half of the
+// chunk (student dS over the teacher logits, teacher dS over the student ones).
 // The logits are read in pieces of PW columns and each piece's load is issued
 // before the previous piece is computed, so the tensor-memory latency overlaps
 // the arithmetic; the stores of piece p land on columns [p PW/2, (p+1) PW/2),
 // which pieces 0..p have already read, and never on the piece in flight.
 constexpr int kBwdPiece = 8;
 
-// Query-owner chunk (thread = query row; constants per row, keys kb .. kb+31,
-// keys >= lim hidden).
-template <bool TEACHER, bool MASKED, int PW = kBwdPiece>
+// Query-owner chunk (thread = query row; constants per row, keys kb ..
+// kb+CWID-1, keys >= lim hidden).
+template <bool TEACHER, bool MASKED, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, float cs, float Lt, float Ls, float g,
                                          float KL2, int kb, int lim) {
-    constexpr int NP = 32 / PW;
+    constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
@@ -148,12 +150,15 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 }
 
 // Key-owner chunk (thread = key row; the logits already carry -LSE / scale, so
-// only g and KL log2(e) per query column come from `cst`, two queries per
-// float4 {g, K, g', K'}; columns q < qmin, relative to the chunk, are hidden).
-template <bool TEACHER, bool MASKED, int PW = kBwdPiece>
-__device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float4 *cst,
-                                          int qmin) {
-    constexpr int NP = 32 / PW;
+// only KL log2(e) per query column comes from shared memory, `ktab`, and g
+// too when it varies per row (G_ROW: `gtab`; else every row uses g_uni).
+// Every thread of the warp reads the same two floats (one 8-byte broadcast
+// load per pair), which keeps this traffic small next to the tensor core's
+// shared-memory reads.  Columns q < qmin, relative to the chunk, are hidden.
+template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece>
+__device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
+                                          const float *gtab, float g_uni, int qmin) {
+    constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
@@ -169,9 +174,10 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int q = PW * pc + k;
-            const float4 e = cst[q >> 1];
+            const float2 K = TEACHER ? *reinterpret_cast<const float2 *>(ktab + q) : make_float2(0.f, 0.f);
+            const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
             ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f, 0.f,
-                                     0.f, e.x, e.z, e.y, e.w, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
+                                     0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
         }
         if constexpr (PW == 8) {
             tmem_st4(at + 4 * pc, ps);
@@ -203,13 +209,21 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *ds
     }
 }
 
-// TMEM column (within a 64-column half of a buffer) of the packed bf16 dS for
-// keys/queries [16 ks, 16 ks + 16): chunk ks/2 keeps its dS in the first 16 of
-// its 32 columns.
-__host__ __device__ constexpr uint32_t ds_col(int ks) { return (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8); }
+// Warpgroup layout of both backward kernels: tiles alternate between two TMEM
+// logit buffers; kBwdParities groups of warpgroups take turns on the tiles
+// (1: every warpgroup works on every tile) and the kBwdHalves warpgroups of a
+// group split a tile's 64 columns into chunks of 64 / kBwdHalves.
+constexpr int kBwdParities = 1;
+constexpr int kBwdHalves = 4;
+constexpr int kBwdChunk = 64 / kBwdHalves;
 
-constexpr int kBwdParities = 2;      // ping-pong: tiles alternate between two TMEM buffers
-constexpr int kBwdHalves = 2;        // warpgroups per parity, each taking 64 / kBwdHalves columns
+// TMEM column (within a 64-column half of a buffer) of the packed bf16 dS for
+// keys/queries [16 ks, 16 ks + 16): chunk c = 16 ks / CW keeps its dS in the
+// first CW/2 of its CW columns.
+template <int CW>
+__host__ __device__ constexpr uint32_t ds_col(int ks) {
+    return (uint32_t)((16 * ks / CW) * CW + (16 * ks % CW) / 2);
+}
 
 // ============================================================================ dK kernel
 template <int DT, int DS, bool TEACHER>
@@ -221,7 +235,7 @@ struct DkvCfg {
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int STAGE_TMA = QT_BYTES + QS_BYTES;
     static constexpr int BIAS_BYTES = BM * 16 * 2;  // [64 queries][16] bf16, unswizzled K-major
-    static constexpr int GK_BYTES = BM * 8;         // float2 {g, KL log2(e)} per query
+    static constexpr int GK_BYTES = BM * 8;         // KL log2(e) per query, then g per query
     static constexpr int BIAS_T = STAGE_TMA, BIAS_S = BIAS_T + BIAS_BYTES, GK = BIAS_S + BIAS_BYTES;
     static constexpr int STAGE_BYTES = ((GK + GK_BYTES + 1023) / 1024) * 1024;
     static constexpr int ONES_BYTES = BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
@@ -352,11 +366,12 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh);
             }
-            float2 *gk = reinterpret_cast<float2 *>(st + C::GK);
+            float *ktab = reinterpret_cast<float *>(st + C::GK), *gtab = ktab + C::BM;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int q = lane + 32 * h;
-                gk[q] = make_float2(c0[h].z, c0[h].w * kLog2eF);
+                ktab[q] = c0[h].w * kLog2eF;
+                gtab[q] = c0[h].z;
                 const uint32_t row = (uint32_t)(q >> 3) * 256u + (uint32_t)(q & 7) * 16u;
                 *reinterpret_cast<uint2 *>(st + C::BIAS_T + row) = split3_bf16(-c0[h].x * p.inv_scale_t);
                 *reinterpret_cast<uint2 *>(st + C::BIAS_S + row) = split3_bf16(-c0[h].y * p.inv_scale_s);
@@ -413,12 +428,12 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BM / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
+                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col<kBwdChunk>(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
                                 (t > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BM / 16; ++ks)
-                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + 64 + ds_col(ks), desc_add(mQt, ks * 2048),
+                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + 64 + ds_col<kBwdChunk>(ks), desc_add(mQt, ks * 2048),
                                     C::IDESC_KT, (t > 0 || ks > 0));
                 }
                 mma_commit(&bar_qempty[s]);
@@ -434,29 +449,31 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const int row = sub * 32 + lane;
         const int gk = k0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
-        const uint32_t bufc = lane_base + par * 128;  // this warpgroup's TMEM buffer
+        constexpr int CW = C::CW;
+        const float g_uni = uniform_g(p);
         bool ok = true;
         for (int t = par; t < n_qt; t += kBwdParities) {
-            const int s = t % C::NSTAGE, n = t / C::NSTAGE;
+            const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
             const int q0 = (first_qt + t) * C::BM;
-            if (!mbar_wait(&bar_sfull[par], (t >> 1) & 1, p.st, abort_v, 16) ||
+            if (!mbar_wait(&bar_sfull[buf], (t >> 1) & 1, p.st, abort_v, 16) ||
                 !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
             tc_fence_after();
-            const float4 *cst = reinterpret_cast<const float4 *>(sQ + s * C::STAGE_BYTES + C::GK);   // {g,K,g',K'}
+            const float *ktab = reinterpret_cast<const float *>(sQ + s * C::STAGE_BYTES + C::GK) + half * CW;
+            const float *gtab = ktab + C::BM;
             const int qmin = gk - off - q0;        // first visible query column (causal)
-#pragma unroll
-            for (int cc = 0; cc < C::CW / 32; ++cc) {
-                const int c = half * (C::CW / 32) + cc;   // chunk of the tile
-                const bool masked = p.causal && (k0 + C::BN - 1 > q0 + c * 32 + off);
-                if (masked)
-                    dkv_chunk<TEACHER, true>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, cst + c * 16, qmin - c * 32);
-                else
-                    dkv_chunk<TEACHER, false>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, cst + c * 16, 0);
+            const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
+            const bool masked = p.causal && (k0 + C::BN - 1 > q0 + half * CW + off);
+            if (masked) {
+                if (p.dkl) dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW);
+                else dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW);
+            } else {
+                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0);
+                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull[par]);
+            if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
         }
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
@@ -625,12 +642,12 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 // dQ_s += dS_s K_s : A = dS_s from TMEM (buffer columns [0,32)), B = K_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
+                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col<kBwdChunk>(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
                                 (kt > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BN / 16; ++ks)
-                        mma_bf16_ts(tmem + C::TMEM_DQT, tmem + buf * 128 + 64 + ds_col(ks), desc_add(mKt, ks * 2048),
+                        mma_bf16_ts(tmem + C::TMEM_DQT, tmem + buf * 128 + 64 + ds_col<kBwdChunk>(ks), desc_add(mKt, ks * 2048),
                                     C::IDESC_QT, (kt > 0 || ks > 0));
                 }
                 mma_commit(&bar_kempty[s]);
@@ -646,7 +663,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         const int row = sub * 32 + lane;
         const int gq = q0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
-        const uint32_t bufc = lane_base + par * 128;
+        constexpr int CW = C::CW;
         float Lt = 0.f, Ls = 0.f, g = 0.f, KL2 = 0.f;
         if (gq < p.N_Q) {
             const size_t r = (size_t)bh * p.N_Q + gq;
@@ -658,22 +675,20 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         const int lim = p.causal ? min(p.N_K, gq + off + 1) : p.N_K;   // first hidden key
         bool ok = true;
         for (int kt = par; kt < n_kt; kt += kBwdParities) {
-            if (!mbar_wait(&bar_sfull[par], (kt >> 1) & 1, p.st, abort_v, 26)) { ok = false; break; }
+            const int buf = kt & 1;
+            if (!mbar_wait(&bar_sfull[buf], (kt >> 1) & 1, p.st, abort_v, 26)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int cc = 0; cc < C::CW / 32; ++cc) {
-                const int c = half * (C::CW / 32) + cc;   // chunk of the tile
-                const int kb = (kt_lo + kt) * C::BN + c * 32;
-                const bool masked = (kb + 32 > p.N_K) || (p.causal && (kb + 31 > q0 + off));
-                if (masked)
-                    dq_chunk<TEACHER, true>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
-                else
-                    dq_chunk<TEACHER, false>(bufc + c * 32, bufc + 64 + c * 32, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
-            }
+            const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
+            const int kb = (kt_lo + kt) * C::BN + half * CW;
+            const bool masked = (kb + CW > p.N_K) || (p.causal && (kb + CW - 1 > q0 + off));
+            if (masked)
+                dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
+            else
+                dq_chunk<TEACHER, false, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull[par]);
+            if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
         }
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();
