@@ -38,12 +38,15 @@
 // every tile, each on its own 16-column chunk, so sixteen warps share the
 // exponentials of a tile while the MMA warp computes the logits of the next
 // tile in the other buffer.  A warpgroup reads its chunk in 8-column pieces
-// and writes the chunk's bf16 dS (8 packed columns) over the first half of
-// the same chunk, which only it reads; the MMA warp then uses those columns
+// and writes the chunk's bf16 dS_s and dS_t (8 packed columns each) over its
+// teacher logits, which only it reads; the MMA warp then uses those columns
 // directly as the A operand of the gradient MMA (tcgen05.mma with A in tensor
-// memory), so dS never touches shared memory.  Because MMAs issued by one
-// thread execute in order, S of tile t+2 can be issued into buffer t & 1 right
-// after the gradient MMA of t.
+// memory), so dS never touches shared memory.  The student half of the buffer
+// is free as soon as every warp has read it, so the student logits of tile
+// t+2 are issued then, during the dS math of tile t; because MMAs issued by
+// one thread execute in order, the teacher logits of t+2 follow right after
+// the gradient MMA of t, which leaves only half of the next logits on the
+// critical path.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -106,24 +109,46 @@ __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float u
 
 // The two chunk routines below turn one CWID-column chunk of a warpgroup's S
 // columns (teacher logits at `at`, student at `as`) into this thread's CWID dS
-// values, written as CWID/2 packed bf16 columns over the first half of the
-// chunk (student dS over the teacher logits, teacher dS over the student ones).
-// The logits are read in pieces of PW columns and each piece's load is issued
-// before the previous piece is computed, so the tensor-memory latency overlaps
-// the arithmetic; the stores of piece p land on columns [p PW/2, (p+1) PW/2),
-// which pieces 0..p have already read, and never on the piece in flight.
+// values.  The logits are read in pieces of PW columns and each piece's load
+// is issued before the previous piece is computed, so the tensor-memory
+// latency overlaps the arithmetic.  As soon as the last piece has landed the
+// warp arrives on `sfree` (its student logits are no longer needed, so the
+// next tile's student logits may overwrite them); once the whole chunk is
+// computed, the packed bf16 dS_s (CWID/2 columns) and dS_t (the next CWID/2)
+// are stored over this chunk's teacher logits, which only this warpgroup
+// reads.
 constexpr int kBwdPiece = 8;
+
+__device__ __forceinline__ void release_student_logits(uint64_t *sfree) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(sfree);
+}
+
+template <bool TEACHER, int CWID>
+__device__ __forceinline__ void store_ds(uint32_t at, const uint32_t (&ps)[CWID / 2], const uint32_t (&pt)[CWID / 2]) {
+    static_assert(CWID == 16 || CWID == 32, "8 or 16 packed columns");
+    if constexpr (CWID == 16) {
+        tmem_st8(at, ps);
+        if (TEACHER) tmem_st8(at + 8, pt);
+    } else {
+        tmem_st16(at, ps);
+        if (TEACHER) tmem_st16(at + 16, pt);
+    }
+}
 
 // Query-owner chunk (thread = query row; constants per row, keys kb ..
 // kb+CWID-1, keys >= lim hidden).
 template <bool TEACHER, bool MASKED, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, float cs, float Lt, float Ls, float g,
-                                         float KL2, int kb, int lim) {
+                                         float KL2, int kb, int lim, uint64_t *sfree) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
+    uint32_t ps[CWID / 2], pt[CWID / 2];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
     tmem_ld_wait_bind(ut[0], us[0]);
+    if (NP == 1) release_student_logits(sfree);
 #pragma unroll
     for (int pc = 0; pc < NP; ++pc) {
         const int cur = pc & 1;
@@ -131,22 +156,18 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
             tmem_ld<PW>(at + PW * (pc + 1), ut[cur ^ 1]);
             tmem_ld<PW>(as + PW * (pc + 1), us[cur ^ 1]);
         }
-        uint32_t ps[PW / 2], pt[PW / 2];
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
-            const int j = kb + PW * pc + k;
+            const int j = kb + PW * pc + k, o = (PW * pc + k) >> 1;
             ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, Lt, Lt, Ls, Ls,
-                                     g, g, KL2, KL2, j < lim, j + 1 < lim, ps[k >> 1], pt[k >> 1]);
+                                     g, g, KL2, KL2, j < lim, j + 1 < lim, ps[o], pt[o]);
         }
-        if constexpr (PW == 8) {
-            tmem_st4(at + 4 * pc, ps);
-            if (TEACHER) tmem_st4(as + 4 * pc, pt);
-        } else {
-            tmem_st8(at + 8 * pc, ps);
-            if (TEACHER) tmem_st8(as + 8 * pc, pt);
+        if (pc + 1 < NP) {
+            tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
+            if (pc + 2 == NP) release_student_logits(sfree);
         }
-        if (pc + 1 < NP) tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
     }
+    store_ds<TEACHER, CWID>(at, ps, pt);
 }
 
 // Key-owner chunk (thread = key row; the logits already carry -LSE / scale, so
@@ -157,12 +178,14 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 // shared-memory reads.  Columns q < qmin, relative to the chunk, are hidden.
 template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
-                                          const float *gtab, float g_uni, int qmin) {
+                                          const float *gtab, float g_uni, int qmin, uint64_t *sfree) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
+    uint32_t ps[CWID / 2], pt[CWID / 2];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
     tmem_ld_wait_bind(ut[0], us[0]);
+    if (NP == 1) release_student_logits(sfree);
 #pragma unroll
     for (int pc = 0; pc < NP; ++pc) {
         const int cur = pc & 1;
@@ -170,24 +193,20 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
             tmem_ld<PW>(at + PW * (pc + 1), ut[cur ^ 1]);
             tmem_ld<PW>(as + PW * (pc + 1), us[cur ^ 1]);
         }
-        uint32_t ps[PW / 2], pt[PW / 2];
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int q = PW * pc + k;
             const float2 K = TEACHER ? *reinterpret_cast<const float2 *>(ktab + q) : make_float2(0.f, 0.f);
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
             ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f, 0.f,
-                                     0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[k >> 1], pt[k >> 1]);
+                                     0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1], pt[q >> 1]);
         }
-        if constexpr (PW == 8) {
-            tmem_st4(at + 4 * pc, ps);
-            if (TEACHER) tmem_st4(as + 4 * pc, pt);
-        } else {
-            tmem_st8(at + 8 * pc, ps);
-            if (TEACHER) tmem_st8(as + 8 * pc, pt);
+        if (pc + 1 < NP) {
+            tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
+            if (pc + 2 == NP) release_student_logits(sfree);
         }
-        if (pc + 1 < NP) tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
     }
+    store_ds<TEACHER, CWID>(at, ps, pt);
 }
 
 // Reads `NCOLS` (a multiple of 16) fp32 accumulator columns of this thread's
@@ -217,13 +236,12 @@ constexpr int kBwdParities = 1;
 constexpr int kBwdHalves = 4;
 constexpr int kBwdChunk = 64 / kBwdHalves;
 
-// TMEM column (within a 64-column half of a buffer) of the packed bf16 dS for
-// keys/queries [16 ks, 16 ks + 16): chunk c = 16 ks / CW keeps its dS in the
-// first CW/2 of its CW columns.
-template <int CW>
-__host__ __device__ constexpr uint32_t ds_col(int ks) {
-    return (uint32_t)((16 * ks / CW) * CW + (16 * ks % CW) / 2);
-}
+// TMEM column (within a buffer) of the packed bf16 dS_s for keys/queries
+// [16 ks, 16 ks + 16): each warpgroup's 16-column chunk of the teacher logits
+// holds its 8 packed dS_s columns, then its 8 packed dS_t columns.
+static_assert(kBwdChunk == 16, "dS layout assumes 16-column chunks");
+__host__ __device__ constexpr uint32_t ds_col_s(int ks) { return (uint32_t)(16 * ks); }
+__host__ __device__ constexpr uint32_t ds_col_t(int ks) { return (uint32_t)(16 * ks + 8); }
 
 // ============================================================================ dK kernel
 template <int DT, int DS, bool TEACHER>
@@ -240,8 +258,11 @@ struct DkvCfg {
     static constexpr int STAGE_BYTES = ((GK + GK_BYTES + 1023) / 1024) * 1024;
     static constexpr int ONES_BYTES = BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
     static constexpr int FIXED = KT_BYTES + KS_BYTES + ONES_BYTES;
-    static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
+    static constexpr int NS_RAW = (224 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
+    // the student logits of tile t+2 are issued before the gradient MMA of
+    // tile t releases its stage, so t+2 must not need that stage
+    static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BM / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -265,6 +286,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
 
     __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
+    __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
     __shared__ uint64_t bar_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -287,6 +309,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
             mbar_init(&bar_dsfull[b], 4 * C::NH);
+            mbar_init(&bar_ssfree[b], 4 * C::NH);
         }
         mbar_init(&bar_done, 1);
         abort_flag = 0;
@@ -397,47 +420,61 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dOnes = plain_desc(smem_u32(sOnes), 128, 256);
         const uint64_t dBias0 = plain_desc(smem_u32(sQ + C::BIAS_T), 128, 256);
         if (elect_one()) {
-            // S^T of tile t into buffer t & 1, each plus its rank-1 bias -LSE / scale
-            auto issue_s = [&](int t) -> bool {
+            // Student S^T of tile t (plus its rank-1 bias -LSE_s / scale_s) into
+            // columns [64, 128) of buffer t & 1, once the tile's Q stage has landed.
+            auto issue_ss = [&](int t) -> bool {
                 const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
                 if (!mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 12)) return false;
                 tc_fence_after();
-                const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES), dQs = desc_add(dQt, C::QT_BYTES);
-                const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES), dBs = desc_add(dBt, C::BIAS_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32),
-                                desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
-                mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
+                const uint64_t dQs = desc_add(dQ0, s * C::STAGE_BYTES + C::QT_BYTES);
+                const uint64_t dBs = desc_add(dBias0, s * C::STAGE_BYTES + C::BIAS_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk)
                     mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32),
                                 desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
                 mma_bf16_ss(tmem + buf * 128 + 64, dOnes, dBs, C::IDESC_S, 1);
-                mma_commit(&bar_sfull[buf]);
                 return true;
             };
+            // Teacher S^T (plus bias) into columns [0, 64), then signal the tile.
+            auto issue_st = [&](int t) {
+                const int s = t % C::NSTAGE, buf = t & 1;
+                const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES);
+                const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < DT / 16; ++kk)
+                    mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32),
+                                desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
+                mma_commit(&bar_sfull[buf]);
+            };
             bool ok = mbar_wait(&bar_k, 0, p.st, abort_v, 14);
-            if (ok && n_qt > 0) ok = issue_s(0);
-            if (ok && n_qt > 1) ok = issue_s(1);
+            for (int t = 0; ok && t < 2 && t < n_qt; ++t) {
+                ok = issue_ss(t);
+                if (ok) issue_st(t);
+            }
             for (int t = 0; ok && t < n_qt; ++t) {
                 const int buf = t & 1, s = t % C::NSTAGE;
+                const bool next = t + 2 < n_qt;
+                // The student logits of tile t+2 go into this buffer as soon as every
+                // warp has read tile t's (they keep their dS in the teacher half).
+                if (next && (!mbar_wait(&bar_ssfree[buf], (t >> 1) & 1, p.st, abort_v, 13) || !issue_ss(t + 2)))
+                    break;
                 if (!mbar_wait(&bar_dsfull[buf], (t >> 1) & 1, p.st, abort_v, 15)) break;
                 tc_fence_after();
                 const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
                 // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BM / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col<kBwdChunk>(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
+                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col_s(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
                                 (t > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BM / 16; ++ks)
-                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + 64 + ds_col<kBwdChunk>(ks), desc_add(mQt, ks * 2048),
+                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + ds_col_t(ks), desc_add(mQt, ks * 2048),
                                     C::IDESC_KT, (t > 0 || ks > 0));
                 }
                 mma_commit(&bar_qempty[s]);
-                if (t + 2 < n_qt && !issue_s(t + 2)) break;
+                if (next) issue_st(t + 2);
             }
             mma_commit(&bar_done);
         }
@@ -463,12 +500,16 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             const int qmin = gk - off - q0;        // first visible query column (causal)
             const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
             const bool masked = p.causal && (k0 + C::BN - 1 > q0 + half * CW + off);
+            uint64_t *sfree = &bar_ssfree[buf];
             if (masked) {
-                if (p.dkl) dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW);
-                else dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW);
+                if (p.dkl)
+                    dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW, sfree);
+                else
+                    dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW,
+                                                        sfree);
             } else {
-                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0);
-                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0);
+                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, sfree);
+                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, sfree);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -507,8 +548,11 @@ struct DqCfg {
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
     static constexpr int FIXED = QT_BYTES + QS_BYTES;
-    static constexpr int NS_RAW = (210 * 1024 - FIXED) / STAGE_BYTES;
+    static constexpr int NS_RAW = (224 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
+    // the student logits of tile t+2 are issued before the gradient MMA of
+    // tile t releases its stage, so t+2 must not need that stage
+    static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BN / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -531,6 +575,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *sK = sQs + C::QS_BYTES;               // stages: K_t, K_s
 
     __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
+    __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
     __shared__ uint64_t bar_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -559,6 +604,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sfull[b], 1);
             mbar_init(&bar_dsfull[b], 4 * C::NH);
+            mbar_init(&bar_ssfree[b], 4 * C::NH);
         }
         mbar_init(&bar_done, 1);
         abort_flag = 0;
@@ -614,44 +660,57 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);          // K-major view of a stage
         const uint64_t dK0mn = sw128_desc(smem_u32(sK), C::KBLK, 1024);   // MN-major view of a stage
         if (elect_one()) {
-            // S of key tile kt into buffer kt & 1
-            auto issue_s = [&](int kt) -> bool {
+            // Student S of key tile kt into columns [64, 128) of buffer kt & 1,
+            // once the tile's K stage has landed.
+            auto issue_ss = [&](int kt) -> bool {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE, buf = kt & 1;
                 if (!mbar_wait(&bar_kfull[s], n & 1, p.st, abort_v, 22)) return false;
                 tc_fence_after();
-                const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES), dKs = desc_add(dKt, C::KT_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32),
-                                desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                const uint64_t dKs = desc_add(dK0, s * C::STAGE_BYTES + C::KT_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk)
                     mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32),
                                 desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
-                mma_commit(&bar_sfull[buf]);
                 return true;
             };
+            // Teacher S into columns [0, 64), then signal the tile.
+            auto issue_st = [&](int kt) {
+                const int s = kt % C::NSTAGE, buf = kt & 1;
+                const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < DT / 16; ++kk)
+                    mma_bf16_ss(tmem + buf * 128, desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32),
+                                desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                mma_commit(&bar_sfull[buf]);
+            };
             bool ok = mbar_wait(&bar_q, 0, p.st, abort_v, 24);
-            if (ok) ok = issue_s(0);
-            if (ok && n_kt > 1) ok = issue_s(1);
+            for (int kt = 0; ok && kt < 2 && kt < n_kt; ++kt) {
+                ok = issue_ss(kt);
+                if (ok) issue_st(kt);
+            }
             for (int kt = 0; ok && kt < n_kt; ++kt) {
                 const int buf = kt & 1, s = kt % C::NSTAGE;
+                const bool next = kt + 2 < n_kt;
+                // the student logits of tile kt+2 go into this buffer as soon as
+                // every warp has read tile kt's (they keep their dS in the teacher half)
+                if (next && (!mbar_wait(&bar_ssfree[buf], (kt >> 1) & 1, p.st, abort_v, 23) || !issue_ss(kt + 2)))
+                    break;
                 if (!mbar_wait(&bar_dsfull[buf], (kt >> 1) & 1, p.st, abort_v, 25)) break;
                 tc_fence_after();
                 const uint64_t mKt = desc_add(dK0mn, s * C::STAGE_BYTES), mKs = desc_add(mKt, C::KT_BYTES);
                 // dQ_s += dS_s K_s : A = dS_s from TMEM (buffer columns [0,32)), B = K_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col<kBwdChunk>(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
+                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col_s(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
                                 (kt > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BN / 16; ++ks)
-                        mma_bf16_ts(tmem + C::TMEM_DQT, tmem + buf * 128 + 64 + ds_col<kBwdChunk>(ks), desc_add(mKt, ks * 2048),
+                        mma_bf16_ts(tmem + C::TMEM_DQT, tmem + buf * 128 + ds_col_t(ks), desc_add(mKt, ks * 2048),
                                     C::IDESC_QT, (kt > 0 || ks > 0));
                 }
                 mma_commit(&bar_kempty[s]);
-                if (kt + 2 < n_kt && !issue_s(kt + 2)) break;
+                if (next) issue_st(kt + 2);
             }
             mma_commit(&bar_done);
         }
@@ -682,9 +741,9 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             const int kb = (kt_lo + kt) * C::BN + half * CW;
             const bool masked = (kb + CW > p.N_K) || (p.causal && (kb + CW - 1 > q0 + off));
             if (masked)
-                dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
+                dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, &bar_ssfree[buf]);
             else
-                dq_chunk<TEACHER, false, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim);
+                dq_chunk<TEACHER, false, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, &bar_ssfree[buf]);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
