@@ -66,6 +66,7 @@ struct BwdParams {
     float inv_scale_t, inv_scale_s;
     float *dq_s, *dq_t, *dk_s, *dk_t;
     float *part_s, *part_t;       // splits > 1: per-split dQ partials [splits][BH*N_Q][d]
+    const void *qt_raw, *kt_raw, *qs_raw, *ks_raw;   // the inputs as plain pointers (rows copied to TMEM)
     DevStatus st;
 };
 
@@ -243,13 +244,50 @@ static_assert(kBwdChunk == 16, "dS layout assumes 16-column chunks");
 __host__ __device__ constexpr uint32_t ds_col_s(int ks) { return (uint32_t)(16 * ks); }
 __host__ __device__ constexpr uint32_t ds_col_t(int ks) { return (uint32_t)(16 * ks + 8); }
 
+// Copies this thread's row of a bf16 [rows][D] tensor into W columns of its
+// TMEM lane (two elements per 32-bit column, lower element in the low half:
+// the layout of an A operand that tcgen05.mma reads from tensor memory).
+// `src` points at the first of the 2W elements, or is null for a row past the
+// end of the tensor, which gets zeros.
+template <int W>
+__device__ __forceinline__ void row_to_tmem(uint32_t taddr, const __nv_bfloat16 *src) {
+    static_assert(W == 8 || W == 16, "8 or 16 columns");
+    uint32_t v[W];
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int k = 0; k < W / 4; ++k) {
+        const uint4 x = src ? __ldg(s4 + k) : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+    }
+    if constexpr (W == 16) tmem_st16(taddr, v); else tmem_st8(taddr, v);
+}
+
+// Every warpgroup copies a quarter of the columns of one resident 128-row
+// operand (rows row0 .. row0+127 of head bh of a [BH, N, D] tensor) into
+// tensor memory at column `col`.  Called by the gradient warpgroups only.
+template <int D>
+__device__ __forceinline__ void resident_to_tmem(uint32_t tmem, uint32_t col, const void *base, int bh, int N, int row0,
+                                                 int wg, int sub, int lane) {
+    constexpr int W = D / 2 / 4;
+    const int r = row0 + sub * 32 + lane;
+    const __nv_bfloat16 *src =
+        r < N ? static_cast<const __nv_bfloat16 *>(base) + ((size_t)bh * N + r) * D + wg * 2 * W : nullptr;
+    row_to_tmem<W>(tmem + ((uint32_t)(sub * 32) << 16) + col + wg * W, src);
+}
+
 // ============================================================================ dK kernel
 template <int DT, int DS, bool TEACHER>
 struct DkvCfg {
     static constexpr int BN = 128, BM = 64;       // keys per CTA, queries per tile
     static constexpr int KBLK = 128 * 128;         // [128 rows][64] bf16 box
     static constexpr int QBLK = 64 * 128;          // [64 rows][64] bf16 box
-    static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
+    // Tensor memory: logit buffers [0, 256), dK_s, dK_t, and, when they fit
+    // (K_TMEM: the student-only and d = 64 cases), this CTA's K_t and K_s rows
+    // as packed bf16, so the logit MMAs read only the Q tile from shared memory.
+    static constexpr uint32_t TMEM_DKS = 256, TMEM_DKT = 256 + DS;
+    static constexpr uint32_t TMEM_KT = TMEM_DKT + (TEACHER ? DT : 0), TMEM_KS = TMEM_KT + DT / 2;
+    static constexpr bool K_TMEM = TMEM_KS + DS / 2 <= 512;
+    static constexpr int KT_BYTES = K_TMEM ? 0 : BN * DT * 2, KS_BYTES = K_TMEM ? 0 : BN * DS * 2;
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int STAGE_TMA = QT_BYTES + QS_BYTES;
     static constexpr int BIAS_BYTES = BM * 16 * 2;  // [64 queries][16] bf16, unswizzled K-major
@@ -269,7 +307,6 @@ struct DkvCfg {
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_KS = idesc_bf16(128, DS, 0, 1);
     static constexpr uint32_t IDESC_KT = idesc_bf16(128, DT, 0, 1);
-    static constexpr uint32_t TMEM_DKS = 256, TMEM_DKT = 256 + DS;
 };
 
 template <int DT, int DS, bool TEACHER>
@@ -337,16 +374,30 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
     volatile int *abort_v = &abort_flag;
+    if constexpr (C::K_TMEM) {
+        if (warp >= 2) {
+            const int wg = (warp - 2) >> 2, sub = warp & 3;
+            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
+            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (TMA + per-query constants)
         if (lane == 0) {
-            prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
-            mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+            prefetch_tmap(&mQt); prefetch_tmap(&mQs);
+            if (!C::K_TMEM) {
+                prefetch_tmap(&mKt); prefetch_tmap(&mKs);
+                mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
 #pragma unroll
-            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+            }
         }
         // Per-query constants of a tile: lane l handles queries l and l + 32.  They
         // are fetched from global memory two tiles ahead into registers, with loads
@@ -407,7 +458,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             DevStatus quick = p.st;
             quick.budget_ns = 50000000ull;
             volatile int never = 0;
-            mbar_wait(&bar_k, 0, quick, &never, 11);
+            if (!C::K_TMEM) mbar_wait(&bar_k, 0, quick, &never, 11);
             for (int t = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); t < issued; ++t)
                 mbar_wait(&bar_qfull[t % C::NSTAGE], (t / C::NSTAGE) & 1, quick, &never, 11);
         }
@@ -429,9 +480,14 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 const uint64_t dQs = desc_add(dQ0, s * C::STAGE_BYTES + C::QT_BYTES);
                 const uint64_t dBs = desc_add(dBias0, s * C::STAGE_BYTES + C::BIAS_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < DS / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32),
-                                desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                for (int kk = 0; kk < DS / 16; ++kk) {
+                    const uint64_t b = desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32);
+                    if constexpr (C::K_TMEM)
+                        mma_bf16_ts(tmem + buf * 128 + 64, tmem + C::TMEM_KS + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
                 mma_bf16_ss(tmem + buf * 128 + 64, dOnes, dBs, C::IDESC_S, 1);
                 return true;
             };
@@ -441,13 +497,18 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES);
                 const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32),
-                                desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                for (int kk = 0; kk < DT / 16; ++kk) {
+                    const uint64_t b = desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32);
+                    if constexpr (C::K_TMEM)
+                        mma_bf16_ts(tmem + buf * 128, tmem + C::TMEM_KT + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
                 mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
                 mma_commit(&bar_sfull[buf]);
             };
-            bool ok = mbar_wait(&bar_k, 0, p.st, abort_v, 14);
+            bool ok = C::K_TMEM || mbar_wait(&bar_k, 0, p.st, abort_v, 14);
             for (int t = 0; ok && t < 2 && t < n_qt; ++t) {
                 ok = issue_ss(t);
                 if (ok) issue_st(t);
@@ -544,7 +605,13 @@ struct DqCfg {
     static constexpr int BM = 128, BN = 64;       // queries per CTA, keys per tile
     static constexpr int QBLK = 128 * 128;         // [128 rows][64] bf16 box
     static constexpr int KBLK = 64 * 128;          // [64 rows][64] bf16 box
-    static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
+    // Tensor memory: logit buffers [0, 256), dQ_s, dQ_t, and, when they fit
+    // (Q_TMEM: the student-only and d = 64 cases), this CTA's Q_t and Q_s rows
+    // as packed bf16, so the logit MMAs read only the K tile from shared memory.
+    static constexpr uint32_t TMEM_DQS = 256, TMEM_DQT = 256 + DS;
+    static constexpr uint32_t TMEM_QT = TMEM_DQT + (TEACHER ? DT : 0), TMEM_QS = TMEM_QT + DT / 2;
+    static constexpr bool Q_TMEM = TMEM_QS + DS / 2 <= 512;
+    static constexpr int QT_BYTES = Q_TMEM ? 0 : BM * DT * 2, QS_BYTES = Q_TMEM ? 0 : BM * DS * 2;
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
     static constexpr int FIXED = QT_BYTES + QS_BYTES;
@@ -559,7 +626,6 @@ struct DqCfg {
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_QS = idesc_bf16(128, DS, 0, 1);
     static constexpr uint32_t IDESC_QT = idesc_bf16(128, DT, 0, 1);
-    static constexpr uint32_t TMEM_DQS = 256, TMEM_DQT = 256 + DS;
 };
 
 template <int DT, int DS, bool TEACHER>
@@ -619,16 +685,30 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
     volatile int *abort_v = &abort_flag;
+    if constexpr (C::Q_TMEM) {
+        if (warp >= 2) {
+            const int wg = (warp - 2) >> 2, sub = warp & 3;
+            resident_to_tmem<DT>(tmem, C::TMEM_QT, p.qt_raw, bh, p.N_Q, q0, wg, sub, lane);
+            resident_to_tmem<DS>(tmem, C::TMEM_QS, p.qs_raw, bh, p.N_Q, q0, wg, sub, lane);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
-            prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
-            mbar_expect_tx(&bar_q, C::QT_BYTES + C::QS_BYTES);
+            prefetch_tmap(&mKt); prefetch_tmap(&mKs);
+            if (!C::Q_TMEM) {
+                prefetch_tmap(&mQt); prefetch_tmap(&mQs);
+                mbar_expect_tx(&bar_q, C::QT_BYTES + C::QS_BYTES);
 #pragma unroll
-            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh);
+                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh);
 #pragma unroll
-            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
+                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
+            }
             int issued = 0;
             for (int kt = 0; kt < n_kt; ++kt) {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
@@ -648,7 +728,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 DevStatus quick = p.st;
                 quick.budget_ns = 50000000ull;
                 volatile int never = 0;
-                mbar_wait(&bar_q, 0, quick, &never, 21);
+                if (!C::Q_TMEM) mbar_wait(&bar_q, 0, quick, &never, 21);
                 for (int kt = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); kt < issued; ++kt)
                     mbar_wait(&bar_kfull[kt % C::NSTAGE], (kt / C::NSTAGE) & 1, quick, &never, 21);
             }
@@ -668,9 +748,14 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 tc_fence_after();
                 const uint64_t dKs = desc_add(dK0, s * C::STAGE_BYTES + C::KT_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < DS / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32),
-                                desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                for (int kk = 0; kk < DS / 16; ++kk) {
+                    const uint64_t b = desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32);
+                    if constexpr (C::Q_TMEM)
+                        mma_bf16_ts(tmem + buf * 128 + 64, tmem + C::TMEM_QS + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
                 return true;
             };
             // Teacher S into columns [0, 64), then signal the tile.
@@ -678,12 +763,17 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 const int s = kt % C::NSTAGE, buf = kt & 1;
                 const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < DT / 16; ++kk)
-                    mma_bf16_ss(tmem + buf * 128, desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32),
-                                desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), C::IDESC_S, kk > 0);
+                for (int kk = 0; kk < DT / 16; ++kk) {
+                    const uint64_t b = desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32);
+                    if constexpr (C::Q_TMEM)
+                        mma_bf16_ts(tmem + buf * 128, tmem + C::TMEM_QT + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128, desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
                 mma_commit(&bar_sfull[buf]);
             };
-            bool ok = mbar_wait(&bar_q, 0, p.st, abort_v, 24);
+            bool ok = C::Q_TMEM || mbar_wait(&bar_q, 0, p.st, abort_v, 24);
             for (int kt = 0; ok && kt < 2 && kt < n_kt; ++kt) {
                 ok = issue_ss(kt);
                 if (ok) issue_st(kt);

@@ -254,6 +254,7 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     p.inv_scale_t = 1.0f / scale_t;
     p.inv_scale_s = 1.0f / scale_s;
     p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
+    p.qt_raw = q_t; p.kt_raw = k_t; p.qs_raw = q_s; p.ks_raw = k_s;
     p.st.word = static_cast<uint32_t *>(workspace);
     p.st.budget_ns = kWaitBudgetNs;
     p.splits = 1;
