@@ -215,6 +215,30 @@ def cpu_baseline(w, target_s: float = 15.0):
                       f"{dt:.1f} s wall, metric FLOPs counted over the rows' visible keys"}
 
 
+# ----------------------------------------------------------------------------- multi-rank helpers
+
+def rank_workload(w, rank: int):
+    """The workload one rank solves: the same shape, its own seed (ranks are
+    independent problems; no data crosses between them)."""
+    return dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank timings (the slowest rank decides)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's FLOPs over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, w):
@@ -348,13 +372,13 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
     # each rank solves its own independent problem (its own seed)
-    wr = dataclasses.replace(w, seed=w.seed + 7919 * rank)
+    wr = rank_workload(w, rank)
     host = [t.pin_memory() for t in inputs.make_inputs(wr)]
     x = [t.to(dev, non_blocking=True) for t in host]
     B, H, NQ, NK, dt_, ds_ = w.B, w.H, w.N_Q, w.N_K, w.d_t, w.d_s
@@ -458,14 +482,12 @@ def main():
     ms_e2e = e0.elapsed_time(e1)
 
     if world > 1:
-        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = tt.tolist()
+        ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], world, dev)
 
     ms_step = ms_total / K
     flops = step_flops(w)
-    value = flops * world / (ms_step * 1e-3) / 1e12
-    e2e_value = flops * world / (ms_e2e / K * 1e-3) / 1e12
+    value = job_throughput(flops, world, ms_step)
+    e2e_value = job_throughput(flops, world, ms_e2e / K)
 
     sustained, burst, peak_src = measured_peak()
     kf = kernel_flops(w)
