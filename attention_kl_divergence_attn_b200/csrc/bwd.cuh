@@ -92,7 +92,11 @@ __device__ __forceinline__ uint2 split3_bf16(float x) {
 
 // dS for two adjacent elements, packed as bf16x2 (lower half = first element).
 // Per-element constants: L (log2-domain LSEs), g and KL*log2(e).
-template <bool TEACHER, bool MASKED>
+// With SCALE_G false the factor g is left out (dS / g is stored): the caller
+// applies g to the accumulated gradient instead, which is exact whenever g is
+// the same for every element the accumulator sums (a uniform g, or the
+// per-row g of the query-owner kernel) and saves two multiplies per element.
+template <bool TEACHER, bool MASKED, bool SCALE_G = true>
 __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float us1, float ct, float cs, float Lt0,
                                         float Lt1, float Ls0, float Ls1, float g0, float g1, float K0, float K1,
                                         bool vis0, bool vis1, uint32_t &ps, uint32_t &pt) {
@@ -104,8 +108,13 @@ __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float u
         P0 = vis0 ? P0 : 0.f; Q0 = vis0 ? Q0 : 0.f;
         P1 = vis1 ? P1 : 0.f; Q1 = vis1 ? Q1 : 0.f;
     }
-    ps = pack_bf16(g0 * (Q0 - P0), g1 * (Q1 - P1));
-    if (TEACHER) pt = pack_bf16((g0 * P0) * ((at0 - as0) - K0), (g1 * P1) * ((at1 - as1) - K1));
+    if (SCALE_G) {
+        ps = pack_bf16(g0 * (Q0 - P0), g1 * (Q1 - P1));
+        if (TEACHER) pt = pack_bf16((g0 * P0) * ((at0 - as0) - K0), (g1 * P1) * ((at1 - as1) - K1));
+    } else {
+        ps = pack_bf16(Q0 - P0, Q1 - P1);
+        if (TEACHER) pt = pack_bf16(P0 * ((at0 - as0) - K0), P1 * ((at1 - as1) - K1));
+    }
 }
 
 // The two chunk routines below turn one CWID-column chunk of a warpgroup's S
@@ -139,7 +148,7 @@ __device__ __forceinline__ void store_ds(uint32_t at, const uint32_t (&ps)[CWID 
 }
 
 // Query-owner chunk (thread = query row; constants per row, keys kb ..
-// kb+CWID-1, keys >= lim hidden).
+// kb+CWID-1, keys >= lim hidden).  The row's g multiplies its dQ at the end.
 template <bool TEACHER, bool MASKED, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, float cs, float Lt, float Ls, float g,
                                          float KL2, int kb, int lim, uint64_t *sfree) {
@@ -160,8 +169,8 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int j = kb + PW * pc + k, o = (PW * pc + k) >> 1;
-            ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, Lt, Lt, Ls, Ls,
-                                     g, g, KL2, KL2, j < lim, j + 1 < lim, ps[o], pt[o]);
+            ds_pair<TEACHER, MASKED, false>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, Lt, Lt,
+                                            Ls, Ls, g, g, KL2, KL2, j < lim, j + 1 < lim, ps[o], pt[o]);
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
@@ -173,7 +182,8 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 
 // Key-owner chunk (thread = key row; the logits already carry -LSE / scale, so
 // only KL log2(e) per query column comes from shared memory, `ktab`, and g
-// too when it varies per row (G_ROW: `gtab`; else every row uses g_uni).
+// too when it varies per row (G_ROW: `gtab`; otherwise g is uniform and the
+// caller applies it to the accumulated dK instead).
 // Every thread of the warp reads the same two floats (one 8-byte broadcast
 // load per pair), which keeps this traffic small next to the tensor core's
 // shared-memory reads.  Columns q < qmin, relative to the chunk, are hidden.
@@ -199,8 +209,9 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
             const int q = PW * pc + k;
             const float2 K = TEACHER ? *reinterpret_cast<const float2 *>(ktab + q) : make_float2(0.f, 0.f);
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
-            ds_pair<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f, 0.f,
-                                     0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1], pt[q >> 1]);
+            ds_pair<TEACHER, MASKED, G_ROW>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,
+                                            0.f, 0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1],
+                                            pt[q >> 1]);
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
@@ -582,8 +593,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             const bool store = gk < p.N_K;
             const size_t r = (size_t)bh * p.N_K + (store ? gk : 0);
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
-            drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s, p.dk_s + r * DS + wg * HS, store);
-            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t, p.dk_t + r * DT + wg * HT, store);
+            const float gs = p.dkl ? 1.f : g_uni;         // a uniform g was left out of dS
+            drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + r * DS + wg * HS, store);
+            if (TEACHER)
+                drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + r * DT + wg * HT, store);
         } else if (n_qt == 0 && gk < p.N_K && wg == 0) {
             const size_t r = (size_t)bh * p.N_K + gk;
             for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
@@ -850,8 +863,9 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 dst_t = p.part_t;
             }
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
-            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s, dst_s + r * DS + wg * HS, store);
-            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t, dst_t + r * DT + wg * HT, store);
+            // the row's g was left out of dS
+            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s * g, dst_s + r * DS + wg * HS, store);
+            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t * g, dst_t + r * DT + wg * HT, store);
         }
     }
 
