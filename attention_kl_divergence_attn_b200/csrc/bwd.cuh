@@ -117,6 +117,33 @@ __device__ __forceinline__ void ds_pair(float ut0, float ut1, float us0, float u
     }
 }
 
+// ds_pair without g (SCALE_G false) on packed fp32 pairs: the same operations
+// in the same order, so the same results, with the element-wise arithmetic
+// issued as f32x2 instructions.  ct2, cs2: splatted scales; nLt2, nLs2: minus
+// the log2-domain LSEs of the two elements (zero where a bias MMA already
+// subtracted them); K2: KL log2(e) of the two elements' rows.
+template <bool TEACHER, bool MASKED>
+__device__ __forceinline__ void ds_pair_x2(float ut0, float ut1, float us0, float us1, uint64_t ct2, uint64_t cs2,
+                                           uint64_t nLt2, uint64_t nLs2, uint64_t K2, bool vis0, bool vis1,
+                                           uint32_t &ps, uint32_t &pt) {
+    const uint64_t at = f2fma(f2pack(ut0, ut1), ct2, nLt2);
+    const uint64_t as = f2fma(f2pack(us0, us1), cs2, nLs2);
+    const float2 a = f2unpack(at), b = f2unpack(as);
+    float P0 = ex2(a.x), P1 = ex2(a.y);
+    float Q0 = ex2(b.x), Q1 = ex2(b.y);
+    if (MASKED) {
+        P0 = vis0 ? P0 : 0.f; Q0 = vis0 ? Q0 : 0.f;
+        P1 = vis1 ? P1 : 0.f; Q1 = vis1 ? Q1 : 0.f;
+    }
+    const uint64_t P = f2pack(P0, P1), Q = f2pack(Q0, Q1);
+    const float2 d = f2unpack(f2sub(Q, P));
+    ps = pack_bf16(d.x, d.y);
+    if (TEACHER) {
+        const float2 e = f2unpack(f2mul(P, f2sub(f2sub(at, as), K2)));
+        pt = pack_bf16(e.x, e.y);
+    }
+}
+
 // The two chunk routines below turn one CWID-column chunk of a warpgroup's S
 // columns (teacher logits at `at`, student at `as`) into this thread's CWID dS
 // values.  The logits are read in pieces of PW columns and each piece's load
@@ -169,8 +196,9 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int j = kb + PW * pc + k, o = (PW * pc + k) >> 1;
-            ds_pair<TEACHER, MASKED, false>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, Lt, Lt,
-                                            Ls, Ls, g, g, KL2, KL2, j < lim, j + 1 < lim, ps[o], pt[o]);
+            ds_pair_x2<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], f2splat(ct),
+                                        f2splat(cs), f2splat(-Lt), f2splat(-Ls), f2splat(KL2), j < lim, j + 1 < lim,
+                                        ps[o], pt[o]);
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
@@ -209,9 +237,14 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
             const int q = PW * pc + k;
             const float2 K = TEACHER ? *reinterpret_cast<const float2 *>(ktab + q) : make_float2(0.f, 0.f);
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
-            ds_pair<TEACHER, MASKED, G_ROW>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,
-                                            0.f, 0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1],
-                                            pt[q >> 1]);
+            if constexpr (G_ROW)
+                ds_pair<TEACHER, MASKED, true>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,
+                                               0.f, 0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1],
+                                               pt[q >> 1]);
+            else
+                ds_pair_x2<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], f2splat(ct),
+                                            f2splat(cs), 0ull, 0ull, f2pack(K.x, K.y), q >= qmin, q + 1 >= qmin,
+                                            ps[q >> 1], pt[q >> 1]);
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
