@@ -396,7 +396,7 @@ def main():
 
     names = ["streamkl_fwd_kernel", "streamkl_mean_kernel", "streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"]
 
-    def step(ev=None):
+    def step(ev=None, x=x):
         if flush is not None:
             flush.zero_()
         if ev is not None:
@@ -458,25 +458,44 @@ def main():
     per_kernel = {n: v / K for n, v in per_kernel.items()}
     code = skl.streamkl_check(stream)
 
-    # end to end through the public API: pinned host inputs -> device, step, loss -> host
+    # End to end through the public API: every step copies its inputs from pinned
+    # host memory to the device and reads the loss back.  The copies run on a
+    # second stream into one of two device input sets, so step k+1's upload
+    # overlaps step k's kernels (both inside the timed region).
     loss_h = torch.empty((), dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host)
+    xs = [x, [torch.empty_like(t) for t in x]]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    used = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for dst, src in zip(x, host):
-            dst.copy_(src, non_blocking=True)
-        step()
-        loss_h.copy_(loss, non_blocking=True)
+    def upload(i):
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(used[i])          # the step that last read set i is done
+            for dst, src in zip(xs[i], host):
+                dst.copy_(src, non_blocking=True)
+            copied[i].record(copy_stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    def e2e_run(n, start=None):
+        if start is not None:
+            copy_stream.wait_event(start)
+        upload(0)
+        for k in range(n):
+            cur = k & 1
+            if k + 1 < n:
+                upload(cur ^ 1)
+            stream.wait_event(copied[cur])
+            step(x=xs[cur])
+            used[cur].record(stream)
+            loss_h.copy_(loss, non_blocking=True)
+
+    e2e_run(args.warmup)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    for _ in range(K):
-        e2e_step()
+    e2e_run(K, start=e0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms_e2e = e0.elapsed_time(e1)
