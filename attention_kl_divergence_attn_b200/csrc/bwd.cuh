@@ -212,8 +212,8 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 // only KL log2(e) per query column comes from shared memory, `ktab`, and g
 // too when it varies per row (G_ROW: `gtab`; otherwise g is uniform and the
 // caller applies it to the accumulated dK instead).
-// Every thread of the warp reads the same two floats (one 8-byte broadcast
-// load per pair), which keeps this traffic small next to the tensor core's
+// Every thread of the warp reads the same floats (4-byte broadcast loads, one
+// wavefront each), which keeps this traffic small next to the tensor core's
 // shared-memory reads.  Columns q < qmin, relative to the chunk, are hidden.
 template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
@@ -235,7 +235,8 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int q = PW * pc + k;
-            const float2 K = TEACHER ? *reinterpret_cast<const float2 *>(ktab + q) : make_float2(0.f, 0.f);
+            const float2 K = TEACHER ? make_float2(ld_shared_f32(ktab + q), ld_shared_f32(ktab + q + 1))
+                                     : make_float2(0.f, 0.f);
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
             if constexpr (G_ROW)
                 ds_pair<TEACHER, MASKED, true>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,

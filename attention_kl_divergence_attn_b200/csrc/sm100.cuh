@@ -332,6 +332,15 @@ __device__ __forceinline__ float lg2(float x) {
     return y;
 }
 
+// One 4-byte shared-memory load that the compiler may not merge with its
+// neighbours: when every thread of a warp reads the same address it costs a
+// single wavefront, where a merged 16-byte broadcast load costs several.
+__device__ __forceinline__ float ld_shared_f32(const float *p) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
