@@ -255,25 +255,6 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
     store_ds<TEACHER, CWID>(at, ps, pt);
 }
 
-// Reads `NCOLS` (a multiple of 16) fp32 accumulator columns of this thread's
-// TMEM lane, scales them and writes them to dst (one row, contiguous) if `store`.
-template <int NCOLS>
-__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool store) {
-#pragma unroll 1
-    for (int c = 0; c < NCOLS / 16; ++c) {
-        float v[16];
-        tmem_ld16(taddr + c * 16, v);
-        tmem_ld_wait();
-        if (store) {
-            float4 *d4 = reinterpret_cast<float4 *>(dst + c * 16);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                d4[k] = make_float4(v[4 * k] * scale, v[4 * k + 1] * scale, v[4 * k + 2] * scale,
-                                    v[4 * k + 3] * scale);
-        }
-    }
-}
-
 // Warpgroup layout of both backward kernels: tiles alternate between two TMEM
 // logit buffers; kBwdParities groups of warpgroups take turns on the tiles
 // (1: every warpgroup works on every tile) and the kBwdHalves warpgroups of a
@@ -281,6 +262,36 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *ds
 constexpr int kBwdParities = 1;
 constexpr int kBwdHalves = 4;
 constexpr int kBwdChunk = 64 / kBwdHalves;
+
+// Writes NCOLS (16 or 32) accumulator columns of this warp's 32 TMEM lanes
+// (rows row0 .. row0+31 of the output, of which the first nvalid exist) to
+// global memory, scaled by `scale` (per thread = per row).  Each thread first
+// puts its row into a padded per-warp staging tile in shared memory (stride
+// NCOLS + 1 floats, so the 32 rows fall into different banks), then the warp
+// stores the tile row-segment by row-segment: consecutive lanes write
+// consecutive floats of one row, so every store is a contiguous 64- or
+// 128-byte run instead of 32 scattered 16-byte pieces.  `dst` points at
+// column 0 of row row0; `ld` is the row stride in floats.
+template <int NCOLS>
+__device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *dst, size_t ld, int nvalid,
+                                           float *stage, int lane) {
+    static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
+    constexpr int SP = NCOLS + 1;
+#pragma unroll
+    for (int c = 0; c < NCOLS; c += 16) {
+        float v[16];
+        tmem_ld16(taddr + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) stage[lane * SP + c + k] = v[k] * scale;
+    }
+    __syncwarp();
+    for (int i = lane; i < nvalid * NCOLS; i += 32) {
+        const int r = i / NCOLS, c = i % NCOLS;
+        dst[(size_t)r * ld + c] = stage[r * SP + c];
+    }
+    __syncwarp();
+}
 
 // TMEM column (within a buffer) of the packed bf16 dS_s for keys/queries
 // [16 ks, 16 ks + 16): each warpgroup's 16-column chunk of the teacher logits
@@ -346,6 +357,7 @@ struct DkvCfg {
     // the student logits of tile t+2 are issued before the gradient MMA of
     // tile t releases its stage, so t+2 must not need that stage
     static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
+    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * 33 * 4, "stage ring doubles as the drain staging area");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BM / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -624,13 +636,18 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         }
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
-            const bool store = gk < p.N_K;
-            const size_t r = (size_t)bh * p.N_K + (store ? gk : 0);
+            // every MMA and TMA copy is done: the stage ring is free for staging
+            float *stage = reinterpret_cast<float *>(sQ) + (warp - 2) * 32 * 33;
+            const int row0 = k0 + sub * 32;
+            const int nvalid = max(0, min(32, p.N_K - row0));
+            const size_t r0 = (size_t)bh * p.N_K + row0;
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
             const float gs = p.dkl ? 1.f : g_uni;         // a uniform g was left out of dS
-            drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + r * DS + wg * HS, store);
+            drain_rows<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + r0 * DS + wg * HS, DS, nvalid,
+                           stage, lane);
             if (TEACHER)
-                drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + r * DT + wg * HT, store);
+                drain_rows<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + r0 * DT + wg * HT, DT,
+                               nvalid, stage, lane);
         } else if (n_qt == 0 && gk < p.N_K && wg == 0) {
             const size_t r = (size_t)bh * p.N_K + gk;
             for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
@@ -667,6 +684,7 @@ struct DqCfg {
     // the student logits of tile t+2 are issued before the gradient MMA of
     // tile t releases its stage, so t+2 must not need that stage
     static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
+    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * 33 * 4, "stage ring doubles as the drain staging area");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BN / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -888,18 +906,24 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         }
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();
-            const bool store = gq < p.N_Q;
-            size_t r = (size_t)bh * p.N_Q + (store ? gq : 0);
+            // every MMA and TMA copy is done: the stage ring is free for staging
+            float *stage = reinterpret_cast<float *>(sK) + (warp - 2) * 32 * 33;
+            const int row0 = q0 + sub * 32;
+            const int nvalid = max(0, min(32, p.N_Q - row0));
+            size_t r0 = (size_t)bh * p.N_Q + row0;
             float *dst_s = p.dq_s, *dst_t = p.dq_t;
             if (p.splits > 1) {             // this split's partial, summed by streamkl_split_sum_kernel
-                r += (size_t)split * p.BH * p.N_Q;
+                r0 += (size_t)split * p.BH * p.N_Q;
                 dst_s = p.part_s;
                 dst_t = p.part_t;
             }
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
             // the row's g was left out of dS
-            drain_row<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s * g, dst_s + r * DS + wg * HS, store);
-            if (TEACHER) drain_row<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t * g, dst_t + r * DT + wg * HT, store);
+            drain_rows<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s * g, dst_s + r0 * DS + wg * HS, DS, nvalid,
+                           stage, lane);
+            if (TEACHER)
+                drain_rows<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t * g, dst_t + r0 * DT + wg * HT, DT, nvalid,
+                               stage, lane);
         }
     }
 
