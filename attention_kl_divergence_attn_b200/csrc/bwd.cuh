@@ -408,6 +408,15 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         mbar_init(&bar_done, 1);
         abort_flag = 0;
         fence_barrier_init();
+        // start the resident K tile right away (its latency overlaps the set-up)
+        if (!C::K_TMEM) {
+            prefetch_tmap(&mKt); prefetch_tmap(&mKs);
+            mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -447,14 +456,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         // ------------------------------------------------------------ producer (TMA + per-query constants)
         if (lane == 0) {
             prefetch_tmap(&mQt); prefetch_tmap(&mQs);
-            if (!C::K_TMEM) {
-                prefetch_tmap(&mKt); prefetch_tmap(&mKs);
-                mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
-#pragma unroll
-                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
-#pragma unroll
-                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
-            }
         }
         // Per-query constants of a tile: lane l handles queries l and l + 32.  They
         // are fetched from global memory two tiles ahead into registers, with loads
@@ -740,6 +741,27 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         mbar_init(&bar_done, 1);
         abort_flag = 0;
         fence_barrier_init();
+        // Start the resident Q tile and the first K stages right away, so that
+        // their latency overlaps the tensor-memory allocation and set-up.
+        prefetch_tmap(&mKt); prefetch_tmap(&mKs);
+        if (!C::Q_TMEM) {
+            prefetch_tmap(&mQt); prefetch_tmap(&mQs);
+            mbar_expect_tx(&bar_q, C::QT_BYTES + C::QS_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
+        }
+        for (int kt = 0; kt < min(C::NSTAGE, n_kt); ++kt) {
+            uint8_t *st = sK + kt * C::STAGE_BYTES;
+            mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b)
+                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b)
+                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -765,17 +787,9 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
-            prefetch_tmap(&mKt); prefetch_tmap(&mKs);
-            if (!C::Q_TMEM) {
-                prefetch_tmap(&mQt); prefetch_tmap(&mQs);
-                mbar_expect_tx(&bar_q, C::QT_BYTES + C::QS_BYTES);
-#pragma unroll
-                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh);
-#pragma unroll
-                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
-            }
-            int issued = 0;
-            for (int kt = 0; kt < n_kt; ++kt) {
+            // Q and the first NSTAGE key tiles were issued during set-up
+            int issued = min(C::NSTAGE, n_kt);
+            for (int kt = issued; kt < n_kt; ++kt) {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
                 if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 21)) break;
                 uint8_t *st = sK + s * C::STAGE_BYTES;

@@ -228,6 +228,24 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         }
         abort_flag = 0;
         fence_barrier_init();
+        // Start the resident Q tile and the first K stages right away, so that
+        // their latency overlaps the tensor-memory allocation and set-up.
+        prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
+        mbar_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh);
+#pragma unroll
+        for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh);
+        for (int kt = 0; kt < min(C::NSTAGE, n_kt); ++kt) {
+            uint8_t *st = sK + kt * C::STAGE_BYTES;
+            mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b)
+                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b)
+                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
@@ -242,14 +260,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
-            prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
-            mbar_expect_tx(&bar_q, C::Q_BYTES);
-#pragma unroll
-            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh);
-#pragma unroll
-            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh);
-            int issued = 0;
-            for (int kt = 0; kt < n_kt; ++kt) {
+            // Q and the first NSTAGE key tiles were issued during set-up
+            int issued = min(C::NSTAGE, n_kt);
+            for (int kt = issued; kt < n_kt; ++kt) {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
                 if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 1)) break;
                 uint8_t *st = sK + s * C::STAGE_BYTES;
@@ -268,6 +281,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 DevStatus quick = p.st;
                 quick.budget_ns = 50000000ull;
                 volatile int never = 0;
+                mbar_wait(&bar_q, 0, quick, &never, 1);
                 for (int kt = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); kt < issued; ++kt)
                     mbar_wait(&bar_kfull[kt % C::NSTAGE], (kt / C::NSTAGE) & 1, quick, &never, 1);
             }
