@@ -214,14 +214,16 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
     const bool want_dk = parts & kPartDK, want_dq = parts & kPartDQ;
-    // the teacher pair of each part must be both given or both absent
-    if (want_dk && want_dq && ((dq_t == nullptr) != (dk_t == nullptr))) return STREAMKL_ERR_INVALID_ARG;
-    const bool teacher = want_dk ? dk_t != nullptr : dq_t != nullptr;
     if (!(dloss == dloss)) return STREAMKL_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     const int BH = B * H;
-    if (want_dk && (!dk_s || (teacher && !dk_t))) return STREAMKL_ERR_INVALID_ARG;
-    if (want_dq && (!dq_s || (teacher && !dq_t))) return STREAMKL_ERR_INVALID_ARG;
+    // Outputs with no elements may be NULL (an empty tensor has no storage).
+    const bool dk_out = want_dk && (long long)BH * N_K > 0, dq_out = want_dq && (long long)BH * N_Q > 0;
+    // the teacher pair of each part must be both given or both absent
+    if (dk_out && dq_out && ((dq_t == nullptr) != (dk_t == nullptr))) return STREAMKL_ERR_INVALID_ARG;
+    const bool teacher = dk_out ? dk_t != nullptr : dq_t != nullptr;
+    if (dk_out && (!dk_s || (teacher && !dk_t))) return STREAMKL_ERR_INVALID_ARG;
+    if (dq_out && (!dq_s || (teacher && !dq_t))) return STREAMKL_ERR_INVALID_ARG;
     if ((long long)BH * N_K == 0) return STREAMKL_OK;       // no keys (so no rows either): nothing to write
     if ((long long)BH * N_Q == 0) {                         // keys but no queries: every dK is zero
         if (want_dk) {

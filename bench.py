@@ -140,9 +140,10 @@ def measured_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the device code (the .cuh files that define the kernels)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_kl_divergence_attn_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(f for f in os.listdir(csrc) if f.endswith(".cuh")):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]

@@ -22,7 +22,8 @@
  *    per-row vectors are fp32 [B, H, N_Q]; gradients are fp32 and shaped like
  *    the tensor they belong to.
  *  - Every pointer is a DEVICE pointer on the current CUDA device, 16-byte
- *    aligned, unless stated otherwise.  Inputs are read only.
+ *    aligned, unless stated otherwise.  Inputs are read only.  A pointer to
+ *    an array with no elements (B*H*N_Q or B*H*N_K zero) may be NULL.
  *  - d_t and d_s must each be 64 or 128 (other sizes: STREAMKL_ERR_UNSUPPORTED).
  *    N_Q, N_K need not be multiples of any tile size.
  *  - causal: key j is visible to query i iff j <= i + (N_K - N_Q) (the mask's
