@@ -5,6 +5,8 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <set>
+#include <utility>
 #include <mutex>
 
 #include <cuda.h>
@@ -78,9 +80,22 @@ streamkl_status check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, in
     return STREAMKL_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device)
+// (the attribute persists), so that later calls, including calls made while a
+// stream is being captured into a CUDA graph, only launch.
+std::mutex g_attr_mutex;
+std::set<std::pair<const void *, int>> g_attr_done;
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorUnknown;
+    const std::pair<const void *, int> key(reinterpret_cast<const void *>(kernel), dev);
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    if (g_attr_done.count(key)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g_attr_done.insert(key);
+    return e;
 }
 
 constexpr int kFwdWarpgroups = 4;
