@@ -56,6 +56,11 @@ def step_flops(w) -> float:
     return per * visible_pairs(w) * w.B * w.H
 
 
+def fwd_flops(w) -> float:
+    """The forward's share of step_flops: 2 (d_t + d_s) per visible pair."""
+    return 2 * (w.d_t + w.d_s) * visible_pairs(w) * w.B * w.H
+
+
 def kernel_flops(w) -> dict:
     """MMA FLOPs each kernel issues per launch (what its tensor pipe executes)."""
     n = visible_pairs(w) * w.B * w.H
@@ -172,29 +177,32 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, n_rows: int, seed: int, cores: int):
-    """Times the fp64 oracle on `n_rows` seeded rows of head (0, 0): forward of
-    those rows plus their full backward (dQ rows and dK contributions).
-    Returns (seconds, metric FLOPs of the sampled (query, key) pairs)."""
+def oracle_sample(w, n_rows: int, seed: int, cores: int, heads: int = 1):
+    """Times the fp64 oracle on `n_rows` seeded rows of each of the first
+    `heads` (batch, head) slices: forward of those rows plus their full backward
+    (dQ rows and dK contributions).  Returns (seconds, metric FLOPs of the
+    sampled (query, key) pairs, rows per head)."""
     import numpy as np
     import oracle
     from attention_kl_divergence_attn_b200 import inputs
-    qt, kt, qs, ks = (t[None, None] for t in inputs.head_inputs(w, 0, 0))
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(w.N_Q, size=min(n_rows, w.N_Q), replace=False)).astype(np.int64)
-    qt, kt, qs, ks = (oracle._f64(x) for x in (qt, kt, qs, ks))
     g = 1.0 / w.rows
-    t0 = time.perf_counter()
-    oracle.rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, rows, nthreads=cores)
-    oracle.bwd_rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, g, rows, teacher=w.teacher_grads,
-                    nthreads=cores)
-    dt = time.perf_counter() - t0
+    dt = 0.0
+    for k in range(heads):
+        b, h = divmod(k % (w.B * w.H), w.H)
+        qt, kt, qs, ks = (oracle._f64(t[None, None]) for t in inputs.head_inputs(w, b, h))
+        t0 = time.perf_counter()
+        oracle.rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, rows, nthreads=cores)
+        oracle.bwd_rows(qt, kt, qs, ks, w.scale_t, w.scale_s, w.causal, g, rows, teacher=w.teacher_grads,
+                        nthreads=cores)
+        dt += time.perf_counter() - t0
     if w.causal:
         pairs = float(np.minimum(w.N_K, rows + (w.N_K - w.N_Q) + 1).sum())
     else:
         pairs = float(len(rows) * w.N_K)
     per = step_flops(w) / (visible_pairs(w) * w.B * w.H)
-    return dt, per * pairs, len(rows)
+    return dt, per * pairs * heads, len(rows)
 
 
 def rows_for(w, seconds: float, cores: int) -> int:
@@ -208,12 +216,23 @@ def rows_for(w, seconds: float, cores: int) -> int:
 
 
 def cpu_baseline(w, target_s: float = 15.0):
+    """The oracle on about `target_s` seconds of the workload: a seeded sample of
+    rows of head (0,0), or whole heads (0,0), (0,1), ... when one head takes
+    less; the full step's time is extrapolated linearly from the sample."""
     cores = cpu_cores()
-    dt, fl, n = oracle_sample(w, rows_for(w, target_s, cores), 3, cores)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} seeded query rows of head (0,0): forward plus full backward "
+    n_rows = rows_for(w, target_s, cores)
+    heads = 1
+    if n_rows >= w.N_Q:                             # one whole head is quick: take several
+        t1, _, _ = oracle_sample(w, w.N_Q, 3, cores)
+        heads = int(max(1, min(w.B * w.H, round(target_s / max(t1, 1e-3)))))
+    dt, fl, n = oracle_sample(w, n_rows, 3, cores, heads)
+    value = fl / dt / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} seeded query rows of each of the first {heads} (batch, head) slice(s): forward plus full backward "
                       f"({'teacher and student' if w.teacher_grads else 'student'} gradients) in fp64, "
-                      f"{dt:.1f} s wall, metric FLOPs counted over the rows' visible keys"}
+                      f"{dt:.1f} s wall, metric FLOPs counted over the rows' visible keys",
+            "gflops": value * 1e3,
+            "extrapolated_full_step_s": step_flops(w) / (value * 1e12)}
 
 
 # ----------------------------------------------------------------------------- multi-rank helpers
@@ -457,6 +476,22 @@ def main():
         for i, n in enumerate(names):
             per_kernel[n] += e[i].elapsed_time(e[i + 1])
     per_kernel = {n: v / K for n, v in per_kernel.items()}
+    # forward (with the loss) and backward on their own: medians over the steps
+    fwd_ms = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+    bwd_ms = statistics.median(e[2].elapsed_time(e[4]) for e in evs)
+    # a plain bf16 GEMM through torch (cuBLAS) in the same run, as a reference rate
+    ga = torch.randn(8192, 8192, device=dev).bfloat16()
+    gb = torch.randn(8192, 8192, device=dev).bfloat16()
+    for _ in range(3):
+        torch.matmul(ga, gb)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(20):
+        torch.matmul(ga, gb)
+    g1.record(stream)
+    torch.cuda.synchronize(dev)
+    cublas_tflops = 2 * 8192 ** 3 * 20 / (g0.elapsed_time(g1) * 1e-3) / 1e12
+    del ga, gb
     code = skl.streamkl_check(stream)
 
     # End to end through the public API: every step copies its inputs from pinned
@@ -538,6 +573,10 @@ def main():
             "kernels": {n: {"ms": per_kernel[n], "share": per_kernel[n] / total_k,
                             "mma_tflops": (kf[n] / (per_kernel[n] * 1e-3) / 1e12) if kf[n] else None}
                         for n in names},
+            "phases": {"fwd_ms_median": fwd_ms, "bwd_ms_median": bwd_ms,
+                       "fwd_tflops": fwd_flops(w) / (fwd_ms * 1e-3) / 1e12,
+                       "bwd_tflops": (flops - fwd_flops(w)) / (bwd_ms * 1e-3) / 1e12},
+            "cublas_bf16_gemm_tflops_same_run": cublas_tflops,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
             "gpu_launches": launches_per_step * K,
