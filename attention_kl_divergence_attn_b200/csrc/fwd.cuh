@@ -185,6 +185,52 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
     Ms = Ms_new;
 }
 
+
+// Fully visible chunk with a lagging maximum: the exponentials are computed
+// against the running maxima M_t, M_s right away (no wait for the chunk
+// maximum), which is exact as long as the chunk's maxima exceed them by at most
+// 8 (log2 units: terms up to 2^8); the chunk maxima are computed alongside and,
+// only if some row of the warp broke that bound, the chunk is redone with the
+// new maxima and a rescale.
+__device__ __forceinline__ void online_chunk_lag(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
+                                                 float &Ms, float &lt, float &ls, float &A) {
+    float m0 = fmax3(ut[0], ut[1], ut[2]), m1 = fmax3(ut[3], ut[4], ut[5]);
+    float n0 = fmax3(us[0], us[1], us[2]), n1 = fmax3(us[3], us[4], us[5]);
+#pragma unroll
+    for (int k = 6; k < 30; k += 4) {
+        m0 = fmax3(m0, ut[k], ut[k + 1]);
+        m1 = fmax3(m1, ut[k + 2], ut[k + 3]);
+        n0 = fmax3(n0, us[k], us[k + 1]);
+        n1 = fmax3(n1, us[k + 2], us[k + 3]);
+    }
+    const float cmt = fmax3(m0, m1, fmaxf(ut[30], ut[31])) * ct;
+    const float cms = fmax3(n0, n1, fmaxf(us[30], us[31])) * cs;
+    const bool fits = (cmt <= Mt + 8.f) && (cms <= Ms + 8.f);
+    if (__all_sync(0xffffffffu, fits)) {
+        const uint64_t ct2 = f2splat(ct), cs2 = f2splat(cs);
+        const uint64_t nMt = f2splat(-Mt), nMs = f2splat(-Ms);
+        uint64_t st[2] = {0ull, 0ull}, ss[2] = {0ull, 0ull}, sa[2] = {0ull, 0ull};
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+            const int j = (k >> 1) & 1;
+            const uint64_t xt = f2fma(f2pack(ut[k], ut[k + 1]), ct2, nMt);
+            const uint64_t xs = f2fma(f2pack(us[k], us[k + 1]), cs2, nMs);
+            const uint64_t et = ex2_pair(xt);
+            const uint64_t es = ex2_pair(xs);
+            st[j] = f2add(st[j], et);
+            ss[j] = f2add(ss[j], es);
+            sa[j] = f2fma(et, f2sub(xt, xs), sa[j]);
+        }
+        const float2 t2 = f2unpack(f2add(st[0], st[1])), s2 = f2unpack(f2add(ss[0], ss[1]));
+        const float2 a2 = f2unpack(f2add(sa[0], sa[1]));
+        lt += t2.x + t2.y;
+        ls += s2.x + s2.y;
+        A += fmaf(Mt - Ms, t2.x + t2.y, a2.x + a2.y);
+    } else {
+        online_chunk(ut, us, ct, cs, Mt, Ms, lt, ls, A);
+    }
+}
+
 template <int DT, int DS, int NWG>
 __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     streamkl_fwd_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
@@ -349,7 +395,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                     }
                     online_chunk_masked(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
                 } else {
-                    online_chunk(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                    online_chunk_lag(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
                 }
             }
             tc_fence_before();
