@@ -186,12 +186,12 @@ __device__ __forceinline__ void online_chunk(float (&ut)[32], float (&us)[32], f
 }
 
 
-// Fully visible chunk with a lagging maximum: the exponentials are computed
-// against the running maxima M_t, M_s right away (no wait for the chunk
-// maximum), which is exact as long as the chunk's maxima exceed them by at most
-// 8 (log2 units: terms up to 2^8); the chunk maxima are computed alongside and,
-// only if some row of the warp broke that bound, the chunk is redone with the
-// new maxima and a rescale.
+// Fully visible chunk with a lagging maximum: when every row of the warp has
+// its chunk maxima at most 8 (log2 units) above its running maxima M_t, M_s,
+// the exponentials are taken against the running maxima unchanged (terms up
+// to 2^8, exact in fp32), which skips the two rescale exponentials and the
+// wait for the updated maxima; otherwise the chunk goes through online_chunk
+// with the exact new maxima.
 __device__ __forceinline__ void online_chunk_lag(float (&ut)[32], float (&us)[32], float ct, float cs, float &Mt,
                                                  float &Ms, float &lt, float &ls, float &A) {
     float m0 = fmax3(ut[0], ut[1], ut[2]), m1 = fmax3(ut[3], ut[4], ut[5]);
