@@ -266,29 +266,39 @@ constexpr int kBwdChunk = 64 / kBwdHalves;
 // Writes NCOLS (16 or 32) accumulator columns of this warp's 32 TMEM lanes
 // (rows row0 .. row0+31 of the output, of which the first nvalid exist) to
 // global memory, scaled by `scale` (per thread = per row).  Each thread first
-// puts its row into a padded per-warp staging tile in shared memory (stride
-// NCOLS + 1 floats, so the 32 rows fall into different banks), then the warp
-// stores the tile row-segment by row-segment: consecutive lanes write
-// consecutive floats of one row, so every store is a contiguous 64- or
-// 128-byte run instead of 32 scattered 16-byte pieces.  `dst` points at
-// column 0 of row row0; `ld` is the row stride in floats.
+// puts its row into a per-warp staging tile in shared memory with 16-byte
+// stores (row stride NCOLS + 4 floats: rows stay 16-byte aligned and the eight
+// rows written by a quarter-warp fall into different banks), then the warp
+// stores the tile with 16-byte loads and stores, 32 / (NCOLS / 4) whole row
+// segments per instruction, so every global store covers complete 64- or
+// 128-byte runs.  `dst` points at column 0 of row row0 and is 16-byte
+// aligned, as is `ld` * 4 bytes, the row stride.
+constexpr int kDrainPad = 4;
+
 template <int NCOLS>
 __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *dst, size_t ld, int nvalid,
                                            float *stage, int lane) {
     static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
-    constexpr int SP = NCOLS + 1;
+    constexpr int SP = NCOLS + kDrainPad, V = NCOLS / 4, RPI = 32 / V;
+    float4 *mine = reinterpret_cast<float4 *>(stage + lane * SP);
 #pragma unroll
     for (int c = 0; c < NCOLS; c += 16) {
         float v[16];
         tmem_ld16(taddr + c, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) stage[lane * SP + c + k] = v[k] * scale;
+        for (int k = 0; k < 4; ++k)
+            mine[c / 4 + k] =
+                make_float4(v[4 * k] * scale, v[4 * k + 1] * scale, v[4 * k + 2] * scale, v[4 * k + 3] * scale);
     }
     __syncwarp();
-    for (int i = lane; i < nvalid * NCOLS; i += 32) {
-        const int r = i / NCOLS, c = i % NCOLS;
-        dst[(size_t)r * ld + c] = stage[r * SP + c];
+    const int rr = lane / V, c4 = (lane % V) * 4;
+#pragma unroll
+    for (int j = 0; j < 32 / RPI; ++j) {
+        const int r = j * RPI + rr;
+        if (r < nvalid)
+            *reinterpret_cast<float4 *>(dst + (size_t)r * ld + c4) =
+                *reinterpret_cast<const float4 *>(stage + r * SP + c4);
     }
     __syncwarp();
 }
@@ -357,7 +367,7 @@ struct DkvCfg {
     // the student logits of tile t+2 are issued before the gradient MMA of
     // tile t releases its stage, so t+2 must not need that stage
     static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
-    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * 33 * 4, "stage ring doubles as the drain staging area");
+    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * (32 + kDrainPad) * 4, "stage ring doubles as the drain staging area");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BM / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -394,47 +404,66 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     const int first_qt = p.causal ? max(0, k0 - off) / C::BM : 0;
     const int n_qt = max(0, n_qt_all - first_qt);
 
-    if (threadIdx.x == 0) {
-        mbar_init(&bar_k, 1);
-        for (int s = 0; s < C::NSTAGE; ++s) {
-            mbar_init(&bar_qfull[s], 1 + 32);      // TMA expect_tx + every producer lane (constants)
-            mbar_init(&bar_qempty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bar_sfull[b], 1);
-            mbar_init(&bar_dsfull[b], 4 * C::NH);
-            mbar_init(&bar_ssfree[b], 4 * C::NH);
-        }
-        mbar_init(&bar_done, 1);
-        abort_flag = 0;
-        fence_barrier_init();
-        // start the resident K tile right away (its latency overlaps the set-up)
-        if (!C::K_TMEM) {
-            prefetch_tmap(&mKt); prefetch_tmap(&mKs);
-            mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+    // Set-up.  Each warp has its own part, and the block barrier below waits
+    // for the slowest: issuing a TMA copy takes a while, so before the barrier
+    // only the copies the first logits need are issued (the resident K tile
+    // and the first Q stage); the producer issues the rest after it.
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_init(&bar_k, 1);
+            for (int s = 0; s < C::NSTAGE; ++s) {
+                mbar_init(&bar_qfull[s], 1 + 32);      // TMA expect_tx + every producer lane (constants)
+                mbar_init(&bar_qempty[s], 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bar_sfull[b], 1);
+                mbar_init(&bar_dsfull[b], 4 * C::NH);
+                mbar_init(&bar_ssfree[b], 4 * C::NH);
+            }
+            mbar_init(&bar_done, 1);
+            abort_flag = 0;
+            fence_barrier_init();
+            if (!C::K_TMEM) {
+                prefetch_tmap(&mKt); prefetch_tmap(&mKs);
+                mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
 #pragma unroll
-            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+            }
+            prefetch_tmap(&mQt); prefetch_tmap(&mQs);
+            if (n_qt > 0) {
+                mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
+#pragma unroll
+                for (int b = 0; b < DT / 64; ++b)
+                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+#pragma unroll
+                for (int b = 0; b < DS / 64; ++b)
+                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+            }
         }
-    }
-    if (warp == 1) {
+    } else if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
         tmem_relinquish();
     }
-    // Unswizzled K-major [rows][16] bf16 layout: row r, K block kb at
-    // (r / 8) * 256 + kb * 128 + (r % 8) * 16.  The ones matrix has 1.0 in K
-    // elements 0..2 of every row; the bias tiles start all zero and the producer
-    // later writes only K elements 0..2 of each row.
-    for (int i = threadIdx.x; i < C::ONES_BYTES / 16; i += blockDim.x) {
-        const bool first_block = ((i >> 3) & 1) == 0;   // 16-byte units: 8 rows per K block
-        *reinterpret_cast<uint4 *>(sOnes + i * 16) =
-            first_block ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    if (warp >= 2 && warp < 6) {
+        // One warpgroup writes the constant MMA operands (and makes them
+        // visible to the tensor core: the proxy fence is costly per warp).
+        // Unswizzled K-major [rows][16] bf16 layout: row r, K block kb at
+        // (r / 8) * 256 + kb * 128 + (r % 8) * 16.  The ones matrix has 1.0 in
+        // K elements 0..2 of every row; the bias tiles start all zero and the
+        // producer later writes only K elements 0..2 of each row.
+        const int tid = threadIdx.x - 64;
+        for (int i = tid; i < C::ONES_BYTES / 16; i += 128) {
+            const bool first_block = ((i >> 3) & 1) == 0;   // 16-byte units: 8 rows per K block
+            *reinterpret_cast<uint4 *>(sOnes + i * 16) =
+                first_block ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int st = 0; st < C::NSTAGE; ++st)
+            for (int i = tid; i < 2 * C::BIAS_BYTES / 16; i += 128)
+                *reinterpret_cast<uint4 *>(sQ + st * C::STAGE_BYTES + C::BIAS_T + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
     }
-    for (int st = 0; st < C::NSTAGE; ++st)
-        for (int i = threadIdx.x; i < 2 * C::BIAS_BYTES / 16; i += blockDim.x)
-            *reinterpret_cast<uint4 *>(sQ + st * C::STAGE_BYTES + C::BIAS_T + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -454,9 +483,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (TMA + per-query constants)
-        if (lane == 0) {
-            prefetch_tmap(&mQt); prefetch_tmap(&mQs);
-        }
         // Per-query constants of a tile: lane l handles queries l and l + 32.  They
         // are fetched from global memory two tiles ahead into registers, with loads
         // the compiler may not move (ld_now), so that their latency overlaps the
@@ -489,7 +515,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             load_consts(t + 2, c2);
             if (n > 0 && !mbar_wait(&bar_qempty[s], (n - 1) & 1, p.st, abort_v, 11)) break;
             uint8_t *st = sQ + s * C::STAGE_BYTES;
-            if (lane == 0) {
+            if (lane == 0 && t > 0) {            // the first stage was issued during set-up
                 mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
@@ -638,7 +664,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
             // every MMA and TMA copy is done: the stage ring is free for staging
-            float *stage = reinterpret_cast<float *>(sQ) + (warp - 2) * 32 * 33;
+            float *stage = reinterpret_cast<float *>(sQ) + (warp - 2) * 32 * (32 + kDrainPad);
             const int row0 = k0 + sub * 32;
             const int nvalid = max(0, min(32, p.N_K - row0));
             const size_t r0 = (size_t)bh * p.N_K + row0;
@@ -685,7 +711,7 @@ struct DqCfg {
     // the student logits of tile t+2 are issued before the gradient MMA of
     // tile t releases its stage, so t+2 must not need that stage
     static_assert(NSTAGE >= 3, "stage ring too shallow for the early student logits");
-    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * 33 * 4, "stage ring doubles as the drain staging area");
+    static_assert(NSTAGE * STAGE_BYTES >= 16 * 32 * (32 + kDrainPad) * 4, "stage ring doubles as the drain staging area");
     static constexpr int SMEM = FIXED + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = kBwdHalves, NWG = kBwdParities * kBwdHalves, CW = BN / NH;
     static constexpr int THREADS = 64 + 128 * NWG;
@@ -741,8 +767,10 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         mbar_init(&bar_done, 1);
         abort_flag = 0;
         fence_barrier_init();
-        // Start the resident Q tile and the first K stages right away, so that
-        // their latency overlaps the tensor-memory allocation and set-up.
+        // Start the resident Q tile and the first K stage right away, so that
+        // their latency overlaps the set-up.  Issuing a TMA copy takes a while
+        // and the set-up barrier waits for this thread, so the producer issues
+        // the other stages after it.
         prefetch_tmap(&mKt); prefetch_tmap(&mKs);
         if (!C::Q_TMEM) {
             prefetch_tmap(&mQt); prefetch_tmap(&mQs);
@@ -752,16 +780,12 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
         }
-        for (int kt = 0; kt < min(C::NSTAGE, n_kt); ++kt) {
-            uint8_t *st = sK + kt * C::STAGE_BYTES;
-            mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
+        mbar_expect_tx(&bar_kfull[0], C::STAGE_BYTES);
 #pragma unroll
-            for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, kt_lo * C::BN, bh);
 #pragma unroll
-            for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
-        }
+        for (int b = 0; b < DS / 64; ++b)
+            tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, kt_lo * C::BN, bh);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -787,8 +811,8 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
-            // Q and the first NSTAGE key tiles were issued during set-up
-            int issued = min(C::NSTAGE, n_kt);
+            // Q and the first key tile were issued during set-up
+            int issued = min(1, n_kt);
             for (int kt = issued; kt < n_kt; ++kt) {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
                 if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 21)) break;
@@ -888,8 +912,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         const int wg = (warp - 2) >> 2;
         const int par = wg % kBwdParities, half = wg / kBwdParities;
         const int sub = warp & 3;
-        const int row = sub * 32 + lane;
-        const int gq = q0 + row;
+        const int gq = q0 + sub * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         constexpr int CW = C::CW;
         float Lt = 0.f, Ls = 0.f, g = 0.f, KL2 = 0.f;
@@ -921,7 +944,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();
             // every MMA and TMA copy is done: the stage ring is free for staging
-            float *stage = reinterpret_cast<float *>(sK) + (warp - 2) * 32 * 33;
+            float *stage = reinterpret_cast<float *>(sK) + (warp - 2) * 32 * (32 + kDrainPad);
             const int row0 = q0 + sub * 32;
             const int nvalid = max(0, min(32, p.N_Q - row0));
             size_t r0 = (size_t)bh * p.N_Q + row0;
