@@ -303,6 +303,34 @@ __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *d
     __syncwarp();
 }
 
+// Writes NCOLS (16 or 32) accumulator columns of this thread's TMEM lane,
+// scaled by `scale`, to its output row at `dst` (when `valid`), straight from
+// registers: 32-byte stores when `dst` is 32-byte aligned (whole sectors),
+// else 16-byte stores.
+template <int NCOLS>
+__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool valid) {
+    static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
+    const bool a32 = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
+#pragma unroll
+    for (int c = 0; c < NCOLS; c += 16) {
+        float v[16];
+        tmem_ld16(taddr + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] *= scale;
+        if (valid) {
+            if (a32) {
+                st_global_v8(dst + c, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+                st_global_v8(dst + c + 8, v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; k += 4)
+                    *reinterpret_cast<float4 *>(dst + c + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            }
+        }
+    }
+}
+
 // TMEM column (within a buffer) of the packed bf16 dS_s for keys/queries
 // [16 ks, 16 ks + 16): each warpgroup's 16-column chunk of the teacher logits
 // holds its 8 packed dS_s columns, then its 8 packed dS_t columns.
@@ -679,6 +707,428 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             const size_t r = (size_t)bh * p.N_K + gk;
             for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
             if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[r * DT + c] = 0.f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Item r of a persistent CTA: items (head, row tile) are numbered heaviest
+// first and dealt out in rounds of gridDim.x, alternately left to right and
+// right to left, so that every CTA gets a similar share of heavy and light
+// items; -1 once this CTA has none left.
+__device__ __forceinline__ int persistent_item(int r, int n_items) {
+    const long long base = (long long)r * gridDim.x;
+    const long long j = base + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+    return j < n_items ? (int)j : -1;
+}
+
+template <int DT, int DS, bool TEACHER>
+__global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
+    streamkl_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
+                            const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
+                            const BwdParams p) {
+    // Persistent form of streamkl_bwd_dkv_kernel: each CTA works through its
+    // items (128 keys of one head each, see persistent_item) one after the
+    // other.  Tiles are counted across
+    // items, so the Q stage ring, the logit buffers and their barriers simply
+    // continue from one item to the next: the next item's Q stages load while
+    // the last tiles of the current one are computed, its resident K rows
+    // load as soon as the current item's last logit MMA has completed, and
+    // its first logits are computed while the gradient warps write out the
+    // current item's dK.
+    using C = DkvCfg<DT, DS, TEACHER>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sKt = smem;
+    uint8_t *sKs = sKt + C::KT_BYTES;
+    uint8_t *sOnes = sKs + C::KS_BYTES;            // rank-1 MMA operand (1, 1, 1, 0, ...)
+    uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
+
+    __shared__ uint64_t bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
+    __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
+    __shared__ uint64_t bar_k;                     // this item's resident K rows are in place
+    __shared__ uint64_t bar_kfree;                 // the item's last logit MMA has completed
+    __shared__ uint64_t bar_done;                  // the item's last gradient MMA has completed
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int off = p.N_K - p.N_Q;
+    const int n_qt_all = (p.N_Q + C::BM - 1) / C::BM;
+    const int n_items = p.BH * p.n_tiles;
+    // item j: key tile j / BH (low key tiles see the most queries), head j % BH
+    auto item_geom = [&](int j, int &k0, int &bh, int &first_qt, int &n_qt) {
+        k0 = (j / p.BH) * C::BN;
+        bh = j % p.BH;
+        first_qt = p.causal ? max(0, k0 - off) / C::BM : 0;
+        n_qt = max(0, n_qt_all - first_qt);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < C::NSTAGE; ++s) {
+                mbar_init(&bar_qfull[s], 1 + 32);      // TMA expect_tx + every producer lane (constants)
+                mbar_init(&bar_qempty[s], 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bar_sfull[b], 1);
+                mbar_init(&bar_dsfull[b], 4 * C::NH);
+                mbar_init(&bar_ssfree[b], 4 * C::NH);
+            }
+            // K rows: one TMA arrival, or (in tensor memory) every gradient warp
+            mbar_init(&bar_k, C::K_TMEM ? 4 * C::NH : 1);
+            mbar_init(&bar_kfree, 1);
+            mbar_init(&bar_done, 1);
+            abort_flag = 0;
+            fence_barrier_init();
+            prefetch_tmap(&mKt); prefetch_tmap(&mKs); prefetch_tmap(&mQt); prefetch_tmap(&mQs);
+            // Start the first item's resident K tile and first Q stage right away,
+            // so that their latency overlaps the set-up (the producer issues the
+            // rest after it; issuing a TMA copy takes a while and the set-up
+            // barrier waits for this thread).
+            int k0, bh, first_qt, n_qt;
+            item_geom(persistent_item(0, n_items), k0, bh, first_qt, n_qt);
+            if (n_qt > 0) {
+                if (!C::K_TMEM) {
+                    mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                }
+                mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
+#pragma unroll
+                for (int b = 0; b < DT / 64; ++b)
+                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+#pragma unroll
+                for (int b = 0; b < DS / 64; ++b)
+                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+            }
+        }
+    } else if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    if (warp >= 2 && warp < 6) {
+        // One warpgroup writes the constant MMA operands (and makes them
+        // visible to the tensor core: the proxy fence is costly per warp).
+        // Unswizzled K-major [rows][16] bf16 layout: row r, K block kb at
+        // (r / 8) * 256 + kb * 128 + (r % 8) * 16.  The ones matrix has 1.0 in
+        // K elements 0..2 of every row; the bias tiles start all zero and the
+        // producer later writes only K elements 0..2 of each row.
+        const int tid = threadIdx.x - 64;
+        for (int i = tid; i < C::ONES_BYTES / 16; i += 128) {
+            const bool first_block = ((i >> 3) & 1) == 0;   // 16-byte units: 8 rows per K block
+            *reinterpret_cast<uint4 *>(sOnes + i * 16) =
+                first_block ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int st = 0; st < C::NSTAGE; ++st)
+            for (int i = tid; i < 2 * C::BIAS_BYTES / 16; i += 128)
+                *reinterpret_cast<uint4 *>(sQ + st * C::STAGE_BYTES + C::BIAS_T + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int *abort_v = &abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (TMA + per-query constants)
+        const float g_all = uniform_g(p);
+        int issued = 0, k_issued = 0;              // Q stages and K tiles issued so far
+        int g0 = 0;                                // this item's first tile, counted across items
+        bool ok = true;
+        for (int r = 0, it = 0; ok; ++r) {
+            const int j = persistent_item(r, n_items);
+            if (j < 0) break;
+            int k0, bh, first_qt, n_qt;
+            item_geom(j, k0, bh, first_qt, n_qt);
+            if (n_qt == 0) continue;
+            // item 0 (when it has tiles): its K tile and first Q stage were issued during set-up
+            const bool pre = r == 0;
+            if (!C::K_TMEM && !pre) {
+                // the previous item's K rows stay until its last logit MMA has completed
+                if (it > 0 && !mbar_wait(&bar_kfree, (it - 1) & 1, p.st, abort_v, 10)) break;
+                if (lane == 0) {
+                    mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                }
+            }
+            if (!C::K_TMEM) ++k_issued;
+            // Per-query constants of a tile: lane l handles queries l and l + 32.
+            // They are fetched from global memory two tiles ahead into registers,
+            // with loads the compiler may not move (ld_now), so that their latency
+            // overlaps the tiles in between instead of stalling the ring.
+            auto load_consts = [&](int t, float4 (&v)[2]) {   // raw {lse_t, lse_s, g, kl}
+                const int q0 = (first_qt + t) * C::BM;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int i = q0 + lane + 32 * h;
+                    v[h] = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
+                    if (t < n_qt && i < p.N_Q) {
+                        const size_t rr = (size_t)bh * p.N_Q + i;
+                        v[h].x = ld_now(p.lse_t + rr);
+                        v[h].y = ld_now(p.lse_s + rr);
+                        v[h].z = p.dkl ? ld_now(p.dkl + rr) : g_all;
+                        v[h].w = ld_now(p.kl + rr);
+                    }
+                }
+            };
+            float4 c0[2], c1[2], c2[2];
+            load_consts(0, c1);
+            load_consts(1, c2);
+            for (int t = 0; t < n_qt; ++t) {
+                const int gg = g0 + t, s = gg % C::NSTAGE, n = gg / C::NSTAGE;
+                const int q0 = (first_qt + t) * C::BM;
+                c0[0] = c1[0]; c0[1] = c1[1];
+                c1[0] = c2[0]; c1[1] = c2[1];
+                load_consts(t + 2, c2);
+                if (n > 0 && !mbar_wait(&bar_qempty[s], (n - 1) & 1, p.st, abort_v, 11)) { ok = false; break; }
+                uint8_t *st = sQ + s * C::STAGE_BYTES;
+                if (lane == 0 && !(pre && t == 0)) {
+                    mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b)
+                        tma_load_3d(st + b * C::QBLK, &mQt, &bar_qfull[s], b * 64, q0, bh);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b)
+                        tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh);
+                }
+                float *ktab = reinterpret_cast<float *>(st + C::GK), *gtab = ktab + C::BM;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int q = lane + 32 * h;
+                    ktab[q] = c0[h].w * kLog2eF;
+                    gtab[q] = c0[h].z;
+                    const uint32_t row = (uint32_t)(q >> 3) * 256u + (uint32_t)(q & 7) * 16u;
+                    *reinterpret_cast<uint2 *>(st + C::BIAS_T + row) = split3_bf16(-c0[h].x * p.inv_scale_t);
+                    *reinterpret_cast<uint2 *>(st + C::BIAS_S + row) = split3_bf16(-c0[h].y * p.inv_scale_s);
+                }
+                fence_proxy_async_smem();          // the bias rows are read by the tensor core
+                mbar_arrive(&bar_qfull[s]);
+                issued = gg + 1;
+            }
+            g0 += n_qt;
+            ++it;
+        }
+        if (*abort_v && lane == 0) {
+            // let the copies in flight land before the CTA's memory is released
+            DevStatus quick = p.st;
+            quick.budget_ns = 50000000ull;
+            volatile int never = 0;
+            if (k_issued > 0) mbar_wait(&bar_k, (k_issued - 1) & 1, quick, &never, 11);
+            for (int t = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); t < issued; ++t)
+                mbar_wait(&bar_qfull[t % C::NSTAGE], (t / C::NSTAGE) & 1, quick, &never, 11);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // Descriptors are built once (warp-uniform) and advanced by constant offsets.
+        const uint64_t dKt = sw128_desc(smem_u32(sKt), 16, 1024), dKs = sw128_desc(smem_u32(sKs), 16, 1024);
+        const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);          // K-major view of a stage
+        const uint64_t dQ0mn = sw128_desc(smem_u32(sQ), C::QBLK, 1024);   // MN-major view of a stage
+        const uint64_t dOnes = plain_desc(smem_u32(sOnes), 128, 256);
+        const uint64_t dBias0 = plain_desc(smem_u32(sQ + C::BIAS_T), 128, 256);
+        if (elect_one()) {
+            // Student S^T of tile gg (plus its rank-1 bias -LSE_s / scale_s) into
+            // columns [64, 128) of buffer gg & 1, once the tile's Q stage has landed.
+            auto issue_ss = [&](int gg) -> bool {
+                const int s = gg % C::NSTAGE, n = gg / C::NSTAGE, buf = gg & 1;
+                if (!mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 12)) return false;
+                tc_fence_after();
+                const uint64_t dQs = desc_add(dQ0, s * C::STAGE_BYTES + C::QT_BYTES);
+                const uint64_t dBs = desc_add(dBias0, s * C::STAGE_BYTES + C::BIAS_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < DS / 16; ++kk) {
+                    const uint64_t b = desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32);
+                    if constexpr (C::K_TMEM)
+                        mma_bf16_ts(tmem + buf * 128 + 64, tmem + C::TMEM_KS + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
+                mma_bf16_ss(tmem + buf * 128 + 64, dOnes, dBs, C::IDESC_S, 1);
+                return true;
+            };
+            // Teacher S^T (plus bias) into columns [0, 64), then signal the tile;
+            // after an item's last logits, signal that its K rows may go.
+            auto issue_st = [&](int gg, bool last) {
+                const int s = gg % C::NSTAGE, buf = gg & 1;
+                const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES);
+                const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < DT / 16; ++kk) {
+                    const uint64_t b = desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32);
+                    if constexpr (C::K_TMEM)
+                        mma_bf16_ts(tmem + buf * 128, tmem + C::TMEM_KT + kk * 8, b, C::IDESC_S, kk > 0);
+                    else
+                        mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
+                                    C::IDESC_S, kk > 0);
+                }
+                mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
+                mma_commit(&bar_sfull[buf]);
+                if (last) mma_commit(&bar_kfree);
+            };
+            bool ok = true;
+            int g0 = 0;
+            for (int r = 0, it = 0; ok; ++r) {
+                const int j = persistent_item(r, n_items);
+                if (j < 0) break;
+                int k0, bh, first_qt, n_qt;
+                item_geom(j, k0, bh, first_qt, n_qt);
+                if (n_qt == 0) continue;
+                if (!mbar_wait(&bar_k, it & 1, p.st, abort_v, 14)) break;
+                // the item's first two tiles; their buffers were last used by the
+                // previous item's last two tiles, whose student logits every warp
+                // must have read (their dS is consumed by MMAs issued earlier)
+                for (int t = 0; t < 2 && t < n_qt; ++t) {
+                    const int gg = g0 + t;
+                    if (gg >= 2 && !mbar_wait(&bar_ssfree[gg & 1], ((gg - 2) >> 1) & 1, p.st, abort_v, 13)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!issue_ss(gg)) { ok = false; break; }
+                    issue_st(gg, t == n_qt - 1);
+                }
+                for (int t = 0; ok && t < n_qt; ++t) {
+                    const int gg = g0 + t, buf = gg & 1, s = gg % C::NSTAGE;
+                    const bool next = t + 2 < n_qt;
+                    // The student logits of tile t+2 go into this buffer as soon as every
+                    // warp has read tile t's (they keep their dS in the teacher half).
+                    if (next && (!mbar_wait(&bar_ssfree[buf], (gg >> 1) & 1, p.st, abort_v, 13) || !issue_ss(gg + 2)))
+                        break;
+                    if (!mbar_wait(&bar_dsfull[buf], (gg >> 1) & 1, p.st, abort_v, 15)) break;
+                    tc_fence_after();
+                    const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
+                    // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
+#pragma unroll
+                    for (int ks = 0; ks < C::BM / 16; ++ks)
+                        mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col_s(ks), desc_add(mQs, ks * 2048),
+                                    C::IDESC_KS, (t > 0 || ks > 0));
+                    if (TEACHER) {
+#pragma unroll
+                        for (int ks = 0; ks < C::BM / 16; ++ks)
+                            mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + ds_col_t(ks), desc_add(mQt, ks * 2048),
+                                        C::IDESC_KT, (t > 0 || ks > 0));
+                    }
+                    mma_commit(&bar_qempty[s]);
+                    if (next) issue_st(gg + 2, t + 2 == n_qt - 1);
+                }
+                if (!ok || *abort_v) break;
+                mma_commit(&bar_done);
+                g0 += n_qt;
+                ++it;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ gradient warpgroups (thread = key)
+        const int wg = (warp - 2) >> 2;
+        const int half = wg;
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        constexpr int CW = C::CW;
+        const float g_uni = uniform_g(p);
+        const float gs = p.dkl ? 1.f : g_uni;             // a uniform g was left out of dS
+        bool ok = true;
+        int g0 = 0;
+        // K rows of the item into tensor memory (K_TMEM), once the previous
+        // item's last logit MMA has completed
+        auto k_to_tmem = [&](int it, int k0, int bh) -> bool {
+            if (it > 0 && !mbar_wait(&bar_kfree, (it - 1) & 1, p.st, abort_v, 18)) return false;
+            tc_fence_after();
+            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
+            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_k);
+            return true;
+        };
+        int it = 0;
+        bool k_ready = false;                      // K_TMEM: this item's K rows already copied
+        for (int r = 0; ok; ++r) {
+            const int j = persistent_item(r, n_items);
+            if (j < 0) break;
+            int k0, bh, first_qt, n_qt;
+            item_geom(j, k0, bh, first_qt, n_qt);
+            const int gk = k0 + row;
+            if (n_qt == 0) {
+                if (gk < p.N_K && wg == 0) {       // no visible query: dK = 0
+                    const size_t rr = (size_t)bh * p.N_K + gk;
+                    for (int c = 0; c < DS; ++c) p.dk_s[rr * DS + c] = 0.f;
+                    if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[rr * DT + c] = 0.f;
+                }
+            } else {
+                if (C::K_TMEM && !k_ready && !k_to_tmem(it, k0, bh)) { ok = false; break; }
+                k_ready = false;
+                for (int t = 0; t < n_qt; ++t) {
+                    const int gg = g0 + t, s = gg % C::NSTAGE, n = gg / C::NSTAGE, buf = gg & 1;
+                    const int q0 = (first_qt + t) * C::BM;
+                    if (!mbar_wait(&bar_sfull[buf], (gg >> 1) & 1, p.st, abort_v, 16) ||
+                        !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
+                    tc_fence_after();
+                    const float *ktab = reinterpret_cast<const float *>(sQ + s * C::STAGE_BYTES + C::GK) + half * CW;
+                    const float *gtab = ktab + C::BM;
+                    const int qmin = gk - off - q0;        // first visible query column (causal)
+                    const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
+                    const bool masked = p.causal && (k0 + C::BN - 1 > q0 + half * CW + off);
+                    uint64_t *sfree = &bar_ssfree[buf];
+                    if (masked) {
+                        if (p.dkl)
+                            dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f,
+                                                               qmin - half * CW, sfree);
+                        else
+                            dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni,
+                                                                qmin - half * CW, sfree);
+                    } else {
+                        if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, sfree);
+                        else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, sfree);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
+                }
+                if (!ok) break;
+                if constexpr (C::K_TMEM) {
+                    // the next item with tiles: its K rows go to tensor memory as soon
+                    // as this item's logits are done
+                    for (int rn = r + 1;; ++rn) {
+                        const int jn = persistent_item(rn, n_items);
+                        if (jn < 0) break;
+                        int k0n, bhn, fqn, nqn;
+                        item_geom(jn, k0n, bhn, fqn, nqn);
+                        if (nqn == 0) continue;
+                        if (!k_to_tmem(it + 1, k0n, bhn)) ok = false;
+                        k_ready = true;
+                        break;
+                    }
+                    if (!ok) break;
+                }
+                if (!mbar_wait(&bar_done, it & 1, p.st, abort_v, 19)) { ok = false; break; }
+                tc_fence_after();
+                // dK rows straight from tensor memory to global memory (the stage
+                // ring already holds the next item's tiles)
+                const bool valid = gk < p.N_K;
+                const size_t grow = (size_t)bh * p.N_K + gk;
+                constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
+                drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + grow * DS + wg * HS, valid);
+                if (TEACHER)
+                    drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + grow * DT + wg * HT, valid);
+                tc_fence_before();
+                g0 += n_qt;
+                ++it;
+            }
         }
     }
 

@@ -52,6 +52,14 @@ __device__ __forceinline__ float ld_now(const float *p) {
     return v;
 }
 
+// 32-byte global store (one whole sector; `p` must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(float *p, float a, float b, float c, float d, float e, float f, float g,
+                                             float h) {
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d),
+                 "f"(e), "f"(f), "f"(g), "f"(h)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

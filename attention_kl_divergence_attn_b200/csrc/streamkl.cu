@@ -176,10 +176,17 @@ streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, co
         if (!make_map(&mqt, q_t, DT, N_Q, BH, CK::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CK::BN) ||
             !make_map(&mqs, q_s, DS, N_Q, BH, CK::BM) || !make_map(&mks, k_s, DS, N_K, BH, CK::BN))
             return STREAMKL_ERR_CUDA;
-        auto kdkv = streamkl_bwd_dkv_kernel<DT, DS, TEACHER>;
-        if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
         p.n_tiles = (N_K + CK::BN - 1) / CK::BN;
-        kdkv<<<(unsigned)((long long)BH * p.n_tiles), CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        const long long items = (long long)BH * p.n_tiles;
+        // When the K rows live in tensor memory the kernel has registers to spare
+        // and the persistent form (one CTA per SM working through its share of
+        // the items, overlapping each item's start with the previous one's end)
+        // is faster; at the register limit (teacher and student K in shared
+        // memory) one CTA per item keeps the inner loop faster.
+        auto kdkv = CK::K_TMEM ? streamkl_bwd_dkv_persistent_kernel<DT, DS, TEACHER> : streamkl_bwd_dkv_kernel<DT, DS, TEACHER>;
+        if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+        const long long grid = CK::K_TMEM ? std::min<long long>(items, std::max(1, sm_count())) : items;
+        kdkv<<<(unsigned)grid, CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
     }
     if (parts & kPartDQ) {
