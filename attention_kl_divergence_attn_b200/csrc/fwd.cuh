@@ -274,15 +274,17 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         }
         abort_flag = 0;
         fence_barrier_init();
-        // Start the resident Q tile and the first K stages right away, so that
+        // Start the resident Q tile and the first K stage right away, so that
         // their latency overlaps the tensor-memory allocation and set-up.
+        // Issuing a TMA copy takes a while and the set-up barrier waits for
+        // this thread, so the producer issues the other stages after it.
         prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
         mbar_expect_tx(&bar_q, C::Q_BYTES);
 #pragma unroll
         for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh);
 #pragma unroll
         for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh);
-        for (int kt = 0; kt < min(C::NSTAGE, n_kt); ++kt) {
+        for (int kt = 0; kt < min(1, n_kt); ++kt) {
             uint8_t *st = sK + kt * C::STAGE_BYTES;
             mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
 #pragma unroll
@@ -306,8 +308,8 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
-            // Q and the first NSTAGE key tiles were issued during set-up
-            int issued = min(C::NSTAGE, n_kt);
+            // Q and the first key tile were issued during set-up
+            int issued = min(1, n_kt);
             for (int kt = issued; kt < n_kt; ++kt) {
                 const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
                 if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 1)) break;
