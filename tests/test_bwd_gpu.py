@@ -63,6 +63,29 @@ def test_bwd_small_shapes(shape, per_row_g):
         assert dqt is None and dkt is None
 
 
+@pytest.mark.parametrize("teacher,per_row_g,causal", [(True, True, True), (False, False, False), (True, False, False)])
+def test_bwd_many_items_per_cta(teacher, per_row_g, causal):
+    # 2 x 8 heads x 16 key tiles = 256 key-owner items for 148 SMs: the persistent key-owner
+    # kernel (K rows in tensor memory: d = 64, or student-only) takes several items per CTA,
+    # so its tile counters, stage ring and barrier phases run across item boundaries
+    B, H, N, d = 2, 8, 2048, 64
+    w = inputs.custom(B=B, H=H, N_Q=N, N_K=N, d_t=d, d_s=d, causal=causal, student="independent",
+                      teacher_std=1.5, student_std=1.5, seed=4242 + int(teacher) + 2 * int(causal))
+    qt, kt, qs, ks = inputs.make_inputs(w)
+    if per_row_g:
+        g = torch.randn(B, H, N, generator=torch.Generator().manual_seed(77)) / (B * H * N)
+        dkl, dloss, g_ref = g.cuda(), 0.0, g.double().numpy()
+    else:
+        dkl, dloss, g_ref = None, 1.0, 1.0 / (B * H * N)
+    dqs, dks, dqt, dkt = gpu_grads(w, cuda(qt, kt, qs, ks), teacher, dkl, dloss)
+    r = oracle.bwd(qt, kt, qs, ks, w.scale_t, w.scale_s, causal, g=g_ref, teacher=teacher)
+    assert_grad(to_np(dks), r[1], "dk_s")
+    assert_grad(to_np(dqs), r[0], "dq_s")
+    if teacher:
+        assert_grad(to_np(dkt), r[3], "dk_t")
+        assert_grad(to_np(dqt), r[2], "dq_t")
+
+
 def test_bwd_self_distillation_gives_zero_grads():
     w = inputs.custom(B=1, H=2, N_Q=256, N_K=256, d_t=128, d_s=128, causal=True, seed=9)
     qt, kt = cuda(*inputs.make_inputs(w)[:2])
