@@ -456,38 +456,69 @@ __global__ void __launch_bounds__(256) streamkl_fwd_merge_kernel(const float *__
 }
 
 // Deterministic reduction of n per-row values: out = (sum / div) * mul (the
-// mean with div = n, mul = 1).  One CTA of kMeanThreads threads, each summing
-// a fixed strided subset in fp64 (16-byte loads, eight in flight per thread
-// when the array is 16-byte aligned), then a fixed-shape tree (warp shuffles,
-// then one warp over the warp sums).  The order of additions depends only on
-// n, so the result is the same run to run.
-constexpr int kMeanThreads = 1024;
+// mean with div = n, mul = 1).  One cluster of kMeanCtas CTAs (a single CTA
+// cannot keep enough loads in flight to read a large array quickly): CTA r
+// sums the r-th of kMeanCtas fixed slices, each thread a fixed strided subset
+// in fp64 (16-byte loads, eight in flight per thread when the array is 16-byte
+// aligned), then a fixed-shape tree (warp shuffles, then one warp over the
+// warp sums); CTA 0 adds the kMeanCtas slice totals in rank order, read from
+// the other CTAs' shared memory.  The order of additions depends only on n
+// (and the alignment), so the result is the same run to run.
+constexpr int kMeanThreads = 1024, kMeanCtas = 8;
 
-__global__ void __launch_bounds__(kMeanThreads) streamkl_mean_kernel(const float *__restrict__ v, long long n,
-                                                                     double div, double mul,
-                                                                     float *__restrict__ out) {
+__device__ __forceinline__ unsigned cluster_rank() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// every thread of every CTA of the cluster; orders shared-memory writes
+// before the barrier with reads after it, across the cluster
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// a double in the shared memory of CTA `rank` of this cluster, at the address
+// `p` has in this CTA
+__device__ __forceinline__ double ld_cluster_f64(const double *p, unsigned rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+__global__ void __cluster_dims__(kMeanCtas, 1, 1) __launch_bounds__(kMeanThreads)
+    streamkl_mean_kernel(const float *__restrict__ v, long long n, double div, double mul, float *__restrict__ out) {
     __shared__ double red[kMeanThreads / 32];
+    __shared__ double part;
+    const unsigned rank = cluster_rank();
     double s = 0.0;
-    long long done = 0;
     if ((reinterpret_cast<uintptr_t>(v) & 15) == 0) {
+        // 16-byte groups [g0, g1) of this slice; the last slice also takes the
+        // elements past the last whole group
         const float4 *v4 = reinterpret_cast<const float4 *>(v);
         const long long n4 = n >> 2;
+        const long long g0 = n4 * rank / kMeanCtas, g1 = n4 * (rank + 1) / kMeanCtas;
         constexpr int U = 8;
-        long long k = threadIdx.x;
-        for (; k + (long long)(U - 1) * kMeanThreads < n4; k += (long long)U * kMeanThreads) {
+        long long k = g0 + threadIdx.x;
+        for (; k + (long long)(U - 1) * kMeanThreads < g1; k += (long long)U * kMeanThreads) {
             float4 x[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) x[u] = __ldg(v4 + k + (long long)u * kMeanThreads);
 #pragma unroll
             for (int u = 0; u < U; ++u) s += ((double)x[u].x + (double)x[u].y) + ((double)x[u].z + (double)x[u].w);
         }
-        for (; k < n4; k += kMeanThreads) {
+        for (; k < g1; k += kMeanThreads) {
             const float4 x = __ldg(v4 + k);
             s += ((double)x.x + (double)x.y) + ((double)x.z + (double)x.w);
         }
-        done = n4 << 2;
+        if (rank == kMeanCtas - 1)
+            for (long long e = (n4 << 2) + threadIdx.x; e < n; e += kMeanThreads) s += (double)v[e];
+    } else {
+        const long long e0 = n * rank / kMeanCtas, e1 = n * (rank + 1) / kMeanCtas;
+        for (long long e = e0 + threadIdx.x; e < e1; e += kMeanThreads) s += (double)v[e];
     }
-    for (long long k = done + threadIdx.x; k < n; k += kMeanThreads) s += (double)v[k];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
@@ -496,8 +527,15 @@ __global__ void __launch_bounds__(kMeanThreads) streamkl_mean_kernel(const float
         s = red[threadIdx.x];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (threadIdx.x == 0) *out = n > 0 ? (float)((s / div) * mul) : 0.f;
+        if (threadIdx.x == 0) part = s;
     }
+    cluster_sync();
+    if (rank == 0 && threadIdx.x == 0) {
+        double total = 0.0;
+        for (unsigned r = 0; r < kMeanCtas; ++r) total += ld_cluster_f64(&part, r);
+        *out = n > 0 ? (float)((total / div) * mul) : 0.f;
+    }
+    cluster_sync();                                // CTA 0 has read every slice total
 }
 
 }  // namespace skl

@@ -391,7 +391,7 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     const int BH = B * H;
     const long long rows = (long long)BH * N_Q;
     if (rows == 0) {
-        if (loss_mean) streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
+        if (loss_mean) streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
         return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
     }
     if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
@@ -425,7 +425,7 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     else st = launch_fwd<64, 128>(mqt, mkt, mqs, mks, p, s);
     if (st != STREAMKL_OK) return st;
     if (loss_mean) {
-        streamkl_mean_kernel<<<1, kMeanThreads, 0, s>>>(kl, rows, (double)rows, 1.0, loss_mean);
+        streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, rows, (double)rows, 1.0, loss_mean);
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
     }
     return STREAMKL_OK;
@@ -474,13 +474,13 @@ streamkl_status streamkl_bwd_dloss_device(const void *q_t, const void *k_t, cons
 
 streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream) {
     if (n_rows < 0 || !loss_mean || (n_rows > 0 && !kl)) return STREAMKL_ERR_INVALID_ARG;
-    streamkl_mean_kernel<<<1, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, (double)n_rows, 1.0, loss_mean);
+    streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, (double)n_rows, 1.0, loss_mean);
     return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
 streamkl_status streamkl_loss_reduce(const float *kl, long long n_rows, double factor, float *out, void *stream) {
     if (n_rows < 0 || !out || (n_rows > 0 && !kl) || !(factor == factor)) return STREAMKL_ERR_INVALID_ARG;
-    streamkl_mean_kernel<<<1, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, 1.0, factor, out);
+    streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, (cudaStream_t)stream>>>(kl, n_rows, 1.0, factor, out);
     return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
 }
 
