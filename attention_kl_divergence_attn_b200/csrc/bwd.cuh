@@ -865,6 +865,19 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 }
             }
             if (!C::K_TMEM) ++k_issued;
+            if (C::K_TMEM && lane == 0) {
+                // the next item's K rows, which the gradient warps copy into tensor
+                // memory from global memory at this item's end: bring them into L2 now
+                const int jn = persistent_item(r + 1, n_items);
+                if (jn >= 0) {
+                    int k0n, bhn, fqn, nqn;
+                    item_geom(jn, k0n, bhn, fqn, nqn);
+                    const int rows = min(C::BN, p.N_K - k0n);
+                    const size_t base = (size_t)bhn * p.N_K + k0n;
+                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.kt_raw) + base * DT, (uint32_t)rows * DT * 2);
+                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.ks_raw) + base * DS, (uint32_t)rows * DS * 2);
+                }
+            }
             // Per-query constants of a tile: lane l handles queries l and l + 32.
             // They are fetched from global memory two tiles ahead into registers,
             // with loads the compiler may not move (ld_now), so that their latency

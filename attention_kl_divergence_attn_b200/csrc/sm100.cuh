@@ -60,6 +60,12 @@ __device__ __forceinline__ void st_global_v8(float *p, float a, float b, float c
                  : "memory");
 }
 
+// Asks L2 to fetch `bytes` (a multiple of 16) of global memory starting at the
+// 16-byte aligned `p`, without waiting (a hint: nothing is written anywhere).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
