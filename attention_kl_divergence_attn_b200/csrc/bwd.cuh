@@ -338,37 +338,6 @@ static_assert(kBwdChunk == 16, "dS layout assumes 16-column chunks");
 __host__ __device__ constexpr uint32_t ds_col_s(int ks) { return (uint32_t)(16 * ks); }
 __host__ __device__ constexpr uint32_t ds_col_t(int ks) { return (uint32_t)(16 * ks + 8); }
 
-// Copies this thread's row of a bf16 [rows][D] tensor into W columns of its
-// TMEM lane (two elements per 32-bit column, lower element in the low half:
-// the layout of an A operand that tcgen05.mma reads from tensor memory).
-// `src` points at the first of the 2W elements, or is null for a row past the
-// end of the tensor, which gets zeros.
-template <int W>
-__device__ __forceinline__ void row_to_tmem(uint32_t taddr, const __nv_bfloat16 *src) {
-    static_assert(W == 8 || W == 16, "8 or 16 columns");
-    uint32_t v[W];
-    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-#pragma unroll
-    for (int k = 0; k < W / 4; ++k) {
-        const uint4 x = src ? __ldg(s4 + k) : make_uint4(0u, 0u, 0u, 0u);
-        v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
-    }
-    if constexpr (W == 16) tmem_st16(taddr, v); else tmem_st8(taddr, v);
-}
-
-// Every warpgroup copies a quarter of the columns of one resident 128-row
-// operand (rows row0 .. row0+127 of head bh of a [BH, N, D] tensor) into
-// tensor memory at column `col`.  Called by the gradient warpgroups only.
-template <int D>
-__device__ __forceinline__ void resident_to_tmem(uint32_t tmem, uint32_t col, const void *base, int bh, int N, int row0,
-                                                 int wg, int sub, int lane) {
-    constexpr int W = D / 2 / 4;
-    const int r = row0 + sub * 32 + lane;
-    const __nv_bfloat16 *src =
-        r < N ? static_cast<const __nv_bfloat16 *>(base) + ((size_t)bh * N + r) * D + wg * 2 * W : nullptr;
-    row_to_tmem<W>(tmem + ((uint32_t)(sub * 32) << 16) + col + wg * W, src);
-}
-
 // ============================================================================ dK kernel
 template <int DT, int DS, bool TEACHER>
 struct DkvCfg {

@@ -6,15 +6,21 @@
 // coupled two-distribution KL reduction, so neither softmax is materialised.
 //
 // One CTA owns 128 query rows of one (batch, head).  Roles (2 + 4*NWG warps):
-//   warp 0      TMA producer: Q_t, Q_s once; K_t, K_s tiles of 64 keys into
-//               an NSTAGE-deep shared-memory ring.
+//   warp 0      TMA producer: K_t, K_s tiles of 64 keys into an NSTAGE-deep
+//               shared-memory ring.
 //   warp 1      MMA issuer (one elected thread) and TMEM owner: per key tile
 //               S_t = Q_t K_t^T and S_s = Q_s K_s^T as tcgen05.mma (bf16 in,
-//               fp32 accumulate) into one of four TMEM buffers (4 x 128 cols).
+//               fp32 accumulate) into one of three TMEM buffers (3 x 128 cols).
+//               Q_t and Q_s sit in the last 128 TMEM columns (packed bf16) and
+//               are the MMAs' A operand, so the tensor core reads only the key
+//               tile from shared memory (with both operands from shared memory
+//               an N = 64 MMA is bound by shared-memory bandwidth).
 //   warps 2..   4 softmax warpgroups: 2 parities in ping-pong x 2 column halves.
-//               Warpgroup (p, h) owns key tiles p, p+2, ... (TMEM buffers p and
-//               p+2, so the MMA warp fills a parity's next buffer while it works
-//               on the current one) and, of each, the 32 key columns of half h.
+//               They first copy the CTA's query rows into tensor memory (each
+//               warp a quarter of the columns of its 32 rows).  Warpgroup (p, h)
+//               then owns key tiles p, p+2, ... and, of each, the 32 key columns
+//               of half h; while a parity works on one buffer the MMA warp
+//               fills the next free one.
 //               Four warps per SM sub-partition keep the ex2 unit fed.  Thread = query row
 //               = TMEM lane; it reads its row of both logit tiles in 32-column
 //               chunks (tcgen05.ld 32x32b) and updates its own per-row online
@@ -73,25 +79,51 @@ __device__ __forceinline__ void finish_row(const RowState &x, float *kl, float *
     *kl = LN2 * (x.A / x.lt - lse_t2 + lse_s2);
 }
 
+// Copies warpgroup wg's quarter of one row of a TMA-loaded 128-row bf16 tile
+// (D/64 boxes of [128 rows][64], 128-byte swizzle) into tensor memory at
+// `taddr` (this warp's lane base plus the operand's column): columns
+// wg*W .. wg*W+W-1 of the packed row, W = D/8, two elements per column with
+// the lower element in the low half (the A-operand layout of tcgen05.mma).
+template <int D>
+__device__ __forceinline__ void tile_rows_to_tmem(uint32_t taddr, const uint8_t *tile, int wg, int row) {
+    constexpr int W = D / 2 / 4;
+    uint32_t v[W];
+#pragma unroll
+    for (int k = 0; k < W / 4; ++k) {
+        const int e = wg * 2 * W + k * 8;     // first of the chunk's 8 elements
+        const uint4 x = *reinterpret_cast<const uint4 *>(tile + (e / 64) * (128 * 128) + sw128_offset(row, e % 64));
+        v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+    }
+    if constexpr (W == 16) tmem_st16(taddr + wg * W, v); else tmem_st8(taddr + wg * W, v);
+}
+
+// Deepest key-tile ring the forward uses.
+constexpr int kFwdMaxStages = 4;
+
 template <int DT, int DS, int NWG>
 struct FwdCfg {
     static constexpr int BM = 128, BN = 64;                  // query rows per CTA, keys per tile
     static constexpr int BLK = 128 * 128;                    // one [128 rows][64] bf16 box (Q)
     static constexpr int KBLK = BN * 128;                    // one [64 rows][64] bf16 box (K)
-    static constexpr int NBUF = 4;                           // TMEM logit buffers (S_t, S_s: 64 cols each)
+    static constexpr int NBUF = 3;                           // TMEM logit buffers (S_t, S_s: 64 cols each)
+    // the query tile's rows, packed bf16, after the logit buffers: the logit
+    // MMAs take A from tensor memory and read only the key tile from shared
+    // memory
+    static constexpr uint32_t TMEM_QT = NBUF * 128, TMEM_QS = TMEM_QT + DT / 2;
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int Q_BYTES = QT_BYTES + QS_BYTES;
     static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
     static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
-    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
+    static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > kFwdMaxStages ? kFwdMaxStages : NS_RAW);
     static constexpr int SMEM = Q_BYTES + NSTAGE * STAGE_BYTES + 1024;
     static constexpr int NH = NWG / 2;                       // column halves per parity
     static constexpr int CW = BN / NH;                       // key columns per warpgroup and tile
     static constexpr int THREADS = 64 + 128 * NWG;           // TMA warp, MMA warp, NWG softmax warpgroups
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
-    static_assert(NWG == 2 || NWG == 4, "2 parities x NWG/2 column halves");
+    static_assert(NWG == 4, "2 parities x 2 column halves; four warpgroups copy the query rows");
+    static_assert(TMEM_QS + DS / 2 <= TMEM_COLS, "logit buffers and query rows fit tensor memory");
 };
 
 // Number of key tiles a 128-row query tile starting at q0 must visit.
@@ -239,11 +271,11 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     using C = FwdCfg<DT, DS, NWG>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQt = smem;
+    uint8_t *sQt = smem;                  // landing area of the query rows
     uint8_t *sQs = sQt + C::QT_BYTES;
     uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
 
-    __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
+    __shared__ uint64_t bar_q, bar_qtm, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
@@ -264,6 +296,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bar_q, 1);
+        mbar_init(&bar_qtm, 4 * NWG);    // every softmax warp, once its query rows are in tensor memory
         for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(&bar_kfull[s], 1);
             mbar_init(&bar_kempty[s], 1);
@@ -274,10 +307,10 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         }
         abort_flag = 0;
         fence_barrier_init();
-        // Start the resident Q tile and the first K stage right away, so that
-        // their latency overlaps the tensor-memory allocation and set-up.
-        // Issuing a TMA copy takes a while and the set-up barrier waits for
-        // this thread, so the producer issues the other stages after it.
+        // Start the query tile and the first K stage right away, so that their
+        // latency overlaps the tensor-memory allocation and set-up.  Issuing a
+        // TMA copy takes a while and the set-up barrier waits for this thread,
+        // so the producer issues the other stages after it.
         prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
         mbar_expect_tx(&bar_q, C::Q_BYTES);
 #pragma unroll
@@ -338,10 +371,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         // Descriptors are built once (warp-uniform) and advanced by constant
         // offsets, so the elected thread issues one MMA every few cycles.
-        const uint64_t dQt = sw128_desc(smem_u32(sQt), 16, 1024), dQs = sw128_desc(smem_u32(sQs), 16, 1024);
         const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);
         if (elect_one()) {
-            if (mbar_wait(&bar_q, 0, p.st, abort_v, 2)) {
+            if (mbar_wait(&bar_qtm, 0, p.st, abort_v, 2)) {
                 for (int kt = 0; kt < n_kt; ++kt) {
                     const int s = kt % C::NSTAGE, n = kt / C::NSTAGE;
                     const int buf = kt % C::NBUF, use = kt / C::NBUF;
@@ -352,13 +384,13 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                     const uint32_t dSt = tmem + buf * 128, dSs = dSt + 64;
 #pragma unroll
                     for (int kk = 0; kk < DT / 16; ++kk) {
-                        const uint32_t oq = (kk >> 2) * C::BLK + (kk & 3) * 32, ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
-                        mma_bf16_ss(dSt, desc_add(dQt, oq), desc_add(dKt, ok), C::IDESC, kk > 0);
+                        const uint32_t ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ts(dSt, tmem + C::TMEM_QT + kk * 8, desc_add(dKt, ok), C::IDESC, kk > 0);
                     }
 #pragma unroll
                     for (int kk = 0; kk < DS / 16; ++kk) {
-                        const uint32_t oq = (kk >> 2) * C::BLK + (kk & 3) * 32, ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
-                        mma_bf16_ss(dSs, desc_add(dQs, oq), desc_add(dKs, ok), C::IDESC, kk > 0);
+                        const uint32_t ok = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ts(dSs, tmem + C::TMEM_QS + kk * 8, desc_add(dKs, ok), C::IDESC, kk > 0);
                     }
                     mma_commit(&bar_sfull[buf]);
                     mma_commit(&bar_kempty[s]);
@@ -373,6 +405,15 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         const int row = sub * 32 + lane;
         const int grow = q0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        // this warp's quarter of its 32 rows of Q_t and Q_s into tensor memory
+        if (mbar_wait(&bar_q, 0, p.st, abort_v, 6)) {
+            tile_rows_to_tmem<DT>(lane_base + C::TMEM_QT, sQt, wg, row);
+            tile_rows_to_tmem<DS>(lane_base + C::TMEM_QS, sQs, wg, row);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_qtm);
         float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
         for (int kt = par; kt < n_kt; kt += 2) {
             const int buf = kt % C::NBUF;
