@@ -360,7 +360,8 @@ def workload_config(w) -> dict:
             "causal": w.causal, "teacher_grads": w.teacher_grads, "student": w.student,
             "flops_per_step": step_flops(w),
             "l2": (f"inputs {in_bytes / 1e6:.0f} MB per step vs 126 MB L2; no flush"
-                   if in_bytes > L2_BYTES else "L2 flushed between steps (256 MB write)")}
+                   if in_bytes > L2_BYTES else
+                   "L2 flushed between steps (256 MB write, outside each step's event window)")}
 
 
 # ----------------------------------------------------------------------------- main arm
@@ -471,6 +472,10 @@ def main():
         if world > 1:
             dist.barrier()
     ms_total = t0.elapsed_time(t1)
+    if flush is not None:
+        # the L2 flush runs between steps: time each step from its first to its
+        # last event (the flush before it excluded) and sum over the steps
+        ms_total = sum(e[0].elapsed_time(e[4]) for e in evs)
     per_kernel = {n: 0.0 for n in names}
     for e in evs:
         for i, n in enumerate(names):
