@@ -358,7 +358,16 @@ struct DkvCfg {
     static constexpr int BIAS_T = STAGE_TMA, BIAS_S = BIAS_T + BIAS_BYTES, GK = BIAS_S + BIAS_BYTES;
     static constexpr int STAGE_BYTES = ((GK + GK_BYTES + 1023) / 1024) * 1024;
     static constexpr int ONES_BYTES = BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
-    static constexpr int FIXED = KT_BYTES + KS_BYTES + ONES_BYTES;
+    // K_STAGED (persistent form, K in tensor memory): the next item's K rows
+    // land in a staging area by TMA (K_t boxes, then K_s boxes) and the
+    // gradient warps copy them into tensor memory.  Used when the Q ring keeps
+    // at least five stages beside the area; otherwise the gradient warps read
+    // the rows from global memory (fewer stages cost more than the copy saves).
+    static constexpr int KST_FULL = K_TMEM ? BN * (DT + DS) * 2 : 0;
+    static constexpr bool K_STAGED =
+        K_TMEM && (224 * 1024 - (KT_BYTES + KS_BYTES + ONES_BYTES + KST_FULL)) / STAGE_BYTES >= 5;
+    static constexpr int KST_BYTES = K_STAGED ? KST_FULL : 0;
+    static constexpr int FIXED = KT_BYTES + KS_BYTES + ONES_BYTES + KST_BYTES;
     static constexpr int NS_RAW = (224 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NSTAGE = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
     // the student logits of tile t+2 are issued before the gradient MMA of
@@ -717,13 +726,15 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *sKt = smem;
     uint8_t *sKs = sKt + C::KT_BYTES;
     uint8_t *sOnes = sKs + C::KS_BYTES;            // rank-1 MMA operand (1, 1, 1, 0, ...)
-    uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
+    uint8_t *sKst = sOnes + C::ONES_BYTES;         // K_TMEM: staging area of the next item's K rows
+    uint8_t *sQ = sKst + C::KST_BYTES;             // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
 
     __shared__ uint64_t bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
     __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
     __shared__ uint64_t bar_k;                     // this item's resident K rows are in place
     __shared__ uint64_t bar_kfree;                 // the item's last logit MMA has completed
     __shared__ uint64_t bar_done;                  // the item's last gradient MMA has completed
+    __shared__ uint64_t bar_kst, bar_kstfree;      // K_TMEM: staged K rows landed / copied out
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -754,6 +765,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             mbar_init(&bar_k, C::K_TMEM ? 4 * C::NH : 1);
             mbar_init(&bar_kfree, 1);
             mbar_init(&bar_done, 1);
+            mbar_init(&bar_kst, 1);
+            mbar_init(&bar_kstfree, 4 * C::NH);
             abort_flag = 0;
             fence_barrier_init();
             prefetch_tmap(&mKt); prefetch_tmap(&mKs); prefetch_tmap(&mQt); prefetch_tmap(&mQs);
@@ -770,6 +783,13 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
 #pragma unroll
                     for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                } else if (C::K_STAGED) {
+                    mbar_expect_tx(&bar_kst, C::KST_BYTES);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, k0, bh);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b)
+                        tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, k0, bh);
                 }
                 mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
 #pragma unroll
@@ -814,6 +834,55 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         int issued = 0, k_issued = 0;              // Q stages and K tiles issued so far
         int g0 = 0;                                // this item's first tile, counted across items
         bool ok = true;
+        // K_STAGED: the K rows of the items with tiles pass through the staging
+        // area one item ahead; each copy is issued once the gradient warps have
+        // copied the previous item's rows out of it (checked without blocking
+        // at every Q stage, so the ring keeps filling meanwhile)
+        int kst_r = 0, kst_n = 0;                  // next item to stage: position, index among items with tiles
+        int kst_k0 = 0, kst_bh = 0;
+        bool kst_more = false;                     // such an item exists
+        auto kst_find = [&]() {
+            kst_more = false;
+            for (;; ++kst_r) {
+                const int jj = persistent_item(kst_r, n_items);
+                if (jj < 0) return;
+                int fq, nq;
+                item_geom(jj, kst_k0, kst_bh, fq, nq);
+                if (nq > 0) { kst_more = true; return; }
+            }
+        };
+        auto kst_issue = [&](bool block) -> bool {
+            if (!C::K_STAGED || !kst_more) return true;
+            if (kst_n > 0) {
+                bool fr = lane == 0 && mbar_try_wait(&bar_kstfree, (kst_n - 1) & 1);
+                fr = __shfl_sync(0xffffffffu, fr, 0);
+                if (!fr) {
+                    if (!block) return true;
+                    if (!mbar_wait(&bar_kstfree, (kst_n - 1) & 1, p.st, abort_v, 20)) return false;
+                }
+            }
+            if (lane == 0) {
+                mbar_expect_tx(&bar_kst, C::KST_BYTES);
+#pragma unroll
+                for (int b = 0; b < DT / 64; ++b)
+                    tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kst_bh);
+#pragma unroll
+                for (int b = 0; b < DS / 64; ++b)
+                    tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kst_bh);
+            }
+            ++kst_n;
+            ++kst_r;
+            kst_find();
+            return true;
+        };
+        if constexpr (C::K_STAGED) {
+            kst_find();
+            if (kst_more && kst_r == 0) {          // the first item's rows were issued during set-up
+                ++kst_n;
+                ++kst_r;
+                kst_find();
+            }
+        }
         for (int r = 0, it = 0; ok; ++r) {
             const int j = persistent_item(r, n_items);
             if (j < 0) break;
@@ -834,7 +903,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 }
             }
             if (!C::K_TMEM) ++k_issued;
-            if (C::K_TMEM && lane == 0) {
+            if (C::K_TMEM && !C::K_STAGED && lane == 0) {
                 // the next item's K rows, which the gradient warps copy into tensor
                 // memory from global memory at this item's end: bring them into L2 now
                 const int jn = persistent_item(r + 1, n_items);
@@ -876,6 +945,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 c1[0] = c2[0]; c1[1] = c2[1];
                 load_consts(t + 2, c2);
                 if (n > 0 && !mbar_wait(&bar_qempty[s], (n - 1) & 1, p.st, abort_v, 11)) { ok = false; break; }
+                if (!kst_issue(false)) { ok = false; break; }
                 uint8_t *st = sQ + s * C::STAGE_BYTES;
                 if (lane == 0 && !(pre && t == 0)) {
                     mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
@@ -903,12 +973,15 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             g0 += n_qt;
             ++it;
         }
+        while (ok && kst_more)
+            if (!kst_issue(true)) ok = false;
         if (*abort_v && lane == 0) {
             // let the copies in flight land before the CTA's memory is released
             DevStatus quick = p.st;
             quick.budget_ns = 50000000ull;
             volatile int never = 0;
             if (k_issued > 0) mbar_wait(&bar_k, (k_issued - 1) & 1, quick, &never, 11);
+            if (kst_n > 0) mbar_wait(&bar_kst, (kst_n - 1) & 1, quick, &never, 11);
             for (int t = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); t < issued; ++t)
                 mbar_wait(&bar_qfull[t % C::NSTAGE], (t / C::NSTAGE) & 1, quick, &never, 11);
         }
@@ -1027,13 +1100,23 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         // item's last logit MMA has completed
         auto k_to_tmem = [&](int it, int k0, int bh) -> bool {
             if (it > 0 && !mbar_wait(&bar_kfree, (it - 1) & 1, p.st, abort_v, 18)) return false;
-            tc_fence_after();
-            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
-            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+            if constexpr (C::K_STAGED) {
+                if (!mbar_wait(&bar_kst, it & 1, p.st, abort_v, 21)) return false;
+                tc_fence_after();
+                tile_rows_to_tmem<DT>(lane_base + C::TMEM_KT, sKst, wg, row);
+                tile_rows_to_tmem<DS>(lane_base + C::TMEM_KS, sKst + C::BN * DT * 2, wg, row);
+            } else {
+                tc_fence_after();
+                resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
+                resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_k);
+            if (lane == 0) {
+                if (C::K_STAGED) mbar_arrive(&bar_kstfree);
+                mbar_arrive(&bar_k);
+            }
             return true;
         };
         int it = 0;

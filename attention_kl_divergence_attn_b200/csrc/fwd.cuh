@@ -79,24 +79,6 @@ __device__ __forceinline__ void finish_row(const RowState &x, float *kl, float *
     *kl = LN2 * (x.A / x.lt - lse_t2 + lse_s2);
 }
 
-// Copies warpgroup wg's quarter of one row of a TMA-loaded 128-row bf16 tile
-// (D/64 boxes of [128 rows][64], 128-byte swizzle) into tensor memory at
-// `taddr` (this warp's lane base plus the operand's column): columns
-// wg*W .. wg*W+W-1 of the packed row, W = D/8, two elements per column with
-// the lower element in the low half (the A-operand layout of tcgen05.mma).
-template <int D>
-__device__ __forceinline__ void tile_rows_to_tmem(uint32_t taddr, const uint8_t *tile, int wg, int row) {
-    constexpr int W = D / 2 / 4;
-    uint32_t v[W];
-#pragma unroll
-    for (int k = 0; k < W / 4; ++k) {
-        const int e = wg * 2 * W + k * 8;     // first of the chunk's 8 elements
-        const uint4 x = *reinterpret_cast<const uint4 *>(tile + (e / 64) * (128 * 128) + sw128_offset(row, e % 64));
-        v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
-    }
-    if constexpr (W == 16) tmem_st16(taddr + wg * W, v); else tmem_st8(taddr + wg * W, v);
-}
-
 // Deepest key-tile ring the forward uses.
 constexpr int kFwdMaxStages = 4;
 
