@@ -837,7 +837,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         // K_STAGED: the K rows of the items with tiles pass through the staging
         // area one item ahead; each copy is issued once the gradient warps have
         // copied the previous item's rows out of it (checked without blocking
-        // at every Q stage, so the ring keeps filling meanwhile)
+        // at every Q stage, so the ring keeps filling meanwhile).  Lane 0 alone
+        // keeps this state and issues the copies: no warp-wide step depends on
+        // it, so lanes that leave the loop early on an abort cannot stall it.
         int kst_r = 0, kst_n = 0;                  // next item to stage: position, index among items with tiles
         int kst_k0 = 0, kst_bh = 0;
         bool kst_more = false;                     // such an item exists
@@ -851,31 +853,25 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 if (nq > 0) { kst_more = true; return; }
             }
         };
-        auto kst_issue = [&](bool block) -> bool {
+        auto kst_issue = [&](bool block) -> bool {     // lane 0 only
             if (!C::K_STAGED || !kst_more) return true;
-            if (kst_n > 0) {
-                bool fr = lane == 0 && mbar_try_wait(&bar_kstfree, (kst_n - 1) & 1);
-                fr = __shfl_sync(0xffffffffu, fr, 0);
-                if (!fr) {
-                    if (!block) return true;
-                    if (!mbar_wait(&bar_kstfree, (kst_n - 1) & 1, p.st, abort_v, 20)) return false;
-                }
+            if (kst_n > 0 && !mbar_try_wait(&bar_kstfree, (kst_n - 1) & 1)) {
+                if (!block) return true;
+                if (!mbar_wait(&bar_kstfree, (kst_n - 1) & 1, p.st, abort_v, 20)) return false;
             }
-            if (lane == 0) {
-                mbar_expect_tx(&bar_kst, C::KST_BYTES);
+            mbar_expect_tx(&bar_kst, C::KST_BYTES);
 #pragma unroll
-                for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kst_bh);
+            for (int b = 0; b < DT / 64; ++b)
+                tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kst_bh);
 #pragma unroll
-                for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kst_bh);
-            }
+            for (int b = 0; b < DS / 64; ++b)
+                tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kst_bh);
             ++kst_n;
             ++kst_r;
             kst_find();
             return true;
         };
-        if constexpr (C::K_STAGED) {
+        if (C::K_STAGED && lane == 0) {
             kst_find();
             if (kst_more && kst_r == 0) {          // the first item's rows were issued during set-up
                 ++kst_n;
@@ -945,7 +941,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 c1[0] = c2[0]; c1[1] = c2[1];
                 load_consts(t + 2, c2);
                 if (n > 0 && !mbar_wait(&bar_qempty[s], (n - 1) & 1, p.st, abort_v, 11)) { ok = false; break; }
-                if (!kst_issue(false)) { ok = false; break; }
+                if (lane == 0) kst_issue(false);
                 uint8_t *st = sQ + s * C::STAGE_BYTES;
                 if (lane == 0 && !(pre && t == 0)) {
                     mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
@@ -973,8 +969,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             g0 += n_qt;
             ++it;
         }
-        while (ok && kst_more)
-            if (!kst_issue(true)) ok = false;
+        if (lane == 0)
+            while (ok && kst_more)
+                if (!kst_issue(true)) ok = false;
         if (*abort_v && lane == 0) {
             // let the copies in flight land before the CTA's memory is released
             DevStatus quick = p.st;
