@@ -162,7 +162,10 @@ def recorded_traffic(kernel: str, workload: str):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("source_hash") != kernel_source_hash():
+    # the counters hold for the sources they were taken from, and for later
+    # sources listed with the change that left the captured kernels as they were
+    here = kernel_source_hash()
+    if rec.get("source_hash") != here and here not in {e.get("hash") for e in rec.get("unchanged_for", [])}:
         return None
     e = rec.get("kernels", {}).get(kernel, {})
     if e.get("workload") != workload:
