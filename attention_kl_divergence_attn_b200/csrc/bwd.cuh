@@ -717,7 +717,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     // items, so the Q stage ring, the logit buffers and their barriers simply
     // continue from one item to the next: the next item's Q stages load while
     // the last tiles of the current one are computed, its resident K rows
-    // load as soon as the current item's last logit MMA has completed, and
+    // (already in shared memory by TMA when K_STAGED) go to tensor memory as
+    // soon as the current item's last logit MMA has completed, and
     // its first logits are computed while the gradient warps write out the
     // current item's dK.
     using C = DkvCfg<DT, DS, TEACHER>;
