@@ -80,6 +80,16 @@ streamkl_status check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, in
     return STREAMKL_OK;
 }
 
+// Input and output pointers of the forward: required (and 16-byte aligned)
+// unless the problem has no rows.  Makes no CUDA call.
+streamkl_status fwd_check_pointers(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                                   int N_Q, const float *kl, const float *lse_t, const float *lse_s) {
+    if ((long long)B * H * N_Q == 0) return STREAMKL_OK;
+    if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s)) return STREAMKL_ERR_INVALID_ARG;
+    return STREAMKL_OK;
+}
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device)
 // (the attribute persists), so that later calls, including calls made while a
 // stream is being captured into a CUDA graph, only launch.
@@ -387,6 +397,7 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
     if (st != STREAMKL_OK) return st;
     if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
+    if ((st = fwd_check_pointers(q_t, k_t, q_s, k_s, B, H, N_Q, kl, lse_t, lse_s)) != STREAMKL_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     const int BH = B * H;
     const long long rows = (long long)BH * N_Q;
@@ -394,8 +405,6 @@ streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, 
         if (loss_mean) streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
         return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
     }
-    if (!q_t || !k_t || !q_s || !k_s || !kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
-    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s)) return STREAMKL_ERR_INVALID_ARG;
     if ((st = check_device()) != STREAMKL_OK) return st;
 
     CUtensorMap mqt, mkt, mqs, mks;
@@ -501,23 +510,73 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 256;   // fixed maximum scratch of this entry point
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kMaxDevices] = {};         // device address of the array, per device
+// The array's device address belongs to one CUDA context's copy of this
+// module, so it is cached per context, under the context's unique id (an id
+// is never reused within a process, unlike a context handle, which a new
+// context created after cudaDeviceReset may take over).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Resolves the device address of the static array for the current device
-// (host code cannot use the symbol's name as a device pointer).
+struct CtxFns {
+    CtxGetCurrentFn get_current = nullptr;
+    CtxGetIdFn get_id = nullptr;
+};
+
+const CtxFns &ctx_fns() {
+    static CtxFns fns;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    return fns;
+}
+
+constexpr int kNoAllocCacheSlots = 64;
+std::mutex g_noalloc_mutex;
+unsigned long long g_noalloc_ctx[kNoAllocCacheSlots] = {};   // context ids (0 = free slot)
+void *g_noalloc_ptr[kNoAllocCacheSlots] = {};                // the array's address in that context
+
+// Id of the current context, or 0 if there is none yet.
+bool current_ctx_id(unsigned long long *id) {
+    const CtxFns &f = ctx_fns();
+    if (!f.get_current || !f.get_id) return false;
+    CUcontext ctx = nullptr;
+    if (f.get_current(&ctx) != CUDA_SUCCESS) return false;
+    *id = 0;
+    return !ctx || f.get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Resolves the device address of the static array in the current context
+// (host code cannot use the symbol's name as a device pointer).  The first
+// lookup in a context calls cudaGetSymbolAddress, which also creates the
+// device's primary context when no context is current yet.
 streamkl_status noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return STREAMKL_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return STREAMKL_ERR_UNSUPPORTED;
+    unsigned long long id = 0;
+    if (!current_ctx_id(&id)) return STREAMKL_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return STREAMKL_ERR_CUDA;
-        g_noalloc_ptr[dev] = ptr;
-    }
-    *out = g_noalloc_ptr[dev];
+    for (int k = 0; id && k < kNoAllocCacheSlots; ++k)
+        if (g_noalloc_ctx[k] == id) {
+            *out = g_noalloc_ptr[k];
+            return STREAMKL_OK;
+        }
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return STREAMKL_ERR_CUDA;
+    if (!id && !current_ctx_id(&id)) return STREAMKL_ERR_CUDA;
+    for (int k = 0; id && k < kNoAllocCacheSlots; ++k)
+        if (g_noalloc_ctx[k] == 0) {              // remember it (a full table only means a lookup per call)
+            g_noalloc_ctx[k] = id;
+            g_noalloc_ptr[k] = ptr;
+            break;
+        }
+    *out = ptr;
     return STREAMKL_OK;
 }
 
@@ -530,9 +589,14 @@ extern "C" streamkl_status streamkl_fwd_noalloc(const void *q_t, const void *k_t
     // every problem runs with the minimum workspace (key splitting, which
     // needs more, is only used when the caller's workspace has room for it)
     static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "the array holds the minimum workspace");
-    void *scratch = nullptr;
-    streamkl_status st = noalloc_scratch(&scratch);
+    // Arguments first, with no CUDA call: a rejected call must not clear the
+    // status word that an earlier call, maybe still running, may yet set.
+    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
     if (st != STREAMKL_OK) return st;
+    if ((st = fwd_check_pointers(q_t, k_t, q_s, k_s, B, H, N_Q, kl, lse_t, lse_s)) != STREAMKL_OK) return st;
+    if ((long long)B * H * N_Q > 0 && (st = check_device()) != STREAMKL_OK) return st;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != STREAMKL_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     // the status word must start at zero for this call
     if (cudaMemsetAsync(scratch, 0, kNoAllocScratchBytes, s) != cudaSuccess) return STREAMKL_ERR_CUDA;

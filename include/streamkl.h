@@ -188,12 +188,15 @@ streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int
  * array inside the library (a file-scope __device__ array that every GPU
  * loading the library keeps until the process exits).  Nothing is allocated:
  * no cudaMalloc, no cudaFree, no allocating library call.
- *  - The first call on each device looks up that array's device address
- *    (cudaGetSymbolAddress, with the device current); make that first call
- *    before any stream capture.
- *  - Each call clears the status word at its start.  All calls on a device
- *    share the one array and it keeps the last call's contents, so calls that
- *    overlap on the GPU (different streams, no ordering) race on it.
+ *  - The first call in each CUDA context (for runtime-API callers: once per
+ *    device, in its primary context) looks up that array's device address
+ *    with cudaGetSymbolAddress, with the context current, and caches it under
+ *    the context's unique id; make that first call before any stream capture.
+ *  - Arguments are checked before any CUDA call; a rejected call enqueues
+ *    nothing and leaves the array as it was.  Each accepted call clears the
+ *    status word at its start.  All calls in a context share the one array
+ *    and it keeps the last call's contents, so calls that overlap on the GPU
+ *    (different streams, no ordering) race on it.
  *  - The array holds the 256-byte minimum workspace that every problem runs
  *    with; the forward then does not split key ranges across CTAs (that
  *    needs the larger workspace streamkl_workspace_size reports), so no

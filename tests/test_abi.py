@@ -109,3 +109,19 @@ def test_selftest_argument_errors(L):
     assert L.streamkl_selftest_timeout(None, 256, 10000000, None) == 5
     assert L.streamkl_selftest_timeout(ctypes.c_void_p(16), 256, 10, None) == 1            # budget too short
     assert L.streamkl_selftest_timeout(ctypes.c_void_p(16), 256, 10 ** 10, None) == 1      # above 2 s
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device answer")
+def test_noalloc_checks_arguments_before_any_cuda_call(L):
+    # Without a GPU every CUDA call fails, so a rejected call that answers with
+    # its argument error (not STREAMKL_ERR_CUDA) made no CUDA call first: it
+    # neither resolved nor cleared the library's status array.
+    p = ctypes.c_void_p(16)
+    bad = ctypes.c_void_p(18)
+    fwd = L.streamkl_fwd_noalloc
+    assert fwd(p, p, p, p, 1, 1, 128, 128, 96, 64, 0.1, 0.1, 0, p, p, p, None, None, None) == 2
+    assert fwd(p, p, p, p, 1, 1, 200, 100, 64, 64, 0.1, 0.1, 1, p, p, p, None, None, None) == 1
+    assert fwd(bad, p, p, p, 1, 1, 128, 128, 64, 64, 0.1, 0.1, 0, p, p, p, None, None, None) == 1
+    assert fwd(p, p, p, p, 1, 1, 128, 128, 64, 64, 0.1, 0.1, 0, None, p, p, None, None, None) == 1
+    # a valid call reaches the device check, which fails here
+    assert fwd(p, p, p, p, 1, 1, 128, 128, 64, 64, 0.1, 0.1, 0, p, p, p, None, None, None) == 3
