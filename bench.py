@@ -70,6 +70,18 @@ def kernel_flops(w) -> dict:
             "streamkl_bwd_dq_kernel": (s + g) * n, "streamkl_mean_kernel": 0.0}
 
 
+def kernel_method_flops(w) -> dict:
+    """The method's own FLOPs attributed to each kernel per launch (step_flops
+    split over the kernels): the forward's logits; for each backward kernel its
+    own gradient contraction plus half of the one logit recompute the method
+    counts (the second recompute is this design's duplicate, not the method's)."""
+    n = visible_pairs(w) * w.B * w.H
+    s = 2 * (w.d_t + w.d_s)
+    g = 2 * w.d_s + (2 * w.d_t if w.teacher_grads else 0)
+    return {"streamkl_fwd_kernel": s * n, "streamkl_bwd_dkv_kernel": (s / 2 + g) * n,
+            "streamkl_bwd_dq_kernel": (s / 2 + g) * n, "streamkl_mean_kernel": 0.0}
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -296,54 +308,88 @@ def run_reference(args, w):
 
 # ----------------------------------------------------------------------------- materialised comparison
 
-def run_materialised(args, w):
-    """The computation the fused method replaces, in torch eager on one GPU:
-    both logit matrices and both log-softmax distributions are materialised
-    ([B, H, N_Q, N_K] fp32), the per-row KL is reduced from them and autograd
-    produces the same gradients.  Same FLOP count, so the value compares
-    directly; the peak device memory is reported next to it.  Rank 0 only."""
+_LOGITS_MODE = {}
+
+
+def materialised_logits(a, b):
+    """a [B,H,N,d] @ b[B,H,M,d]^T in fp32 from bf16 inputs: a bf16 GEMM with fp32
+    output where torch has it (with autograd) on this device, else an fp32 GEMM of
+    the upcast inputs (TF32 off), so the logits are fp32 either way."""
     import torch
+    B, H, N, d = a.shape
+    M = b.shape[2]
+    mode = _LOGITS_MODE.get(a.device)
+    if mode is None:
+        mode = "fp32 GEMM"
+        try:
+            t = torch.ones(1, 2, 2, dtype=torch.bfloat16, device=a.device, requires_grad=True)
+            torch.bmm(t, t, out_dtype=torch.float32).sum().backward()
+            mode = "bf16 GEMM, fp32 output"
+        except Exception:
+            pass
+        _LOGITS_MODE[a.device] = mode
+    if mode == "fp32 GEMM":
+        return torch.matmul(a.float(), b.float().transpose(-1, -2))
+    return torch.bmm(a.reshape(B * H, N, d), b.reshape(B * H, M, d).transpose(1, 2),
+                     out_dtype=torch.float32).reshape(B, H, N, M)
+
+
+def materialised_step(x, w, mask=None):
+    """The computation the fused method replaces: both [B, H, N_Q, N_K] logit
+    matrices and both log-softmax distributions materialised in fp32, the
+    per-row KL(P || Q) reduced from them, and autograd through all of it for
+    the gradients of the mean loss (left in x[i].grad).  Returns (kl, loss)."""
     import torch.nn.functional as F
+    for t in x:
+        t.grad = None
+    st = materialised_logits(x[0], x[1]) * w.scale_t
+    ss = materialised_logits(x[2], x[3]) * w.scale_s
+    if mask is not None:                  # finite fill: P = 0 there, and no inf - inf
+        st = st.masked_fill(mask, -1e9)
+        ss = ss.masked_fill(mask, -1e9)
+    logp, logq = F.log_softmax(st, -1), F.log_softmax(ss, -1)
+    kl = F.kl_div(logq, logp, reduction="none", log_target=True).sum(-1)
+    loss = kl.mean()
+    loss.backward()
+    return kl.detach(), loss.detach()
+
+
+def materialised_mask(w, device):
+    """The causal mask (True = hidden) of a workload, or None."""
+    import torch
+    if not w.causal:
+        return None
+    i = torch.arange(w.N_Q, device=device)[:, None]
+    j = torch.arange(w.N_K, device=device)[None, :]
+    return j > i + (w.N_K - w.N_Q)
+
+
+def run_materialised(args, w):
+    """The computation the fused method replaces, in torch eager on one GPU
+    (materialised_step).  Same FLOP count, so the value compares directly; the
+    peak device memory is reported next to it.  Rank 0 only."""
+    import torch
     from attention_kl_divergence_attn_b200 import inputs
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     base = {"impl": "materialised", "metric": METRIC, "unit": "TFLOP/s", "n_gpus": 1,
-            "config": workload_config(w), "data": "synthetic", "dtype": "bf16 matmul, fp32 softmax/KL"}
+            "config": workload_config(w), "data": "synthetic"}
     try:
         x = [t.to(dev) for t in inputs.make_inputs(w)]
         for i, t in enumerate(x):
             t.requires_grad_(i >= 2 or w.teacher_grads)
-        mask = None
-        if w.causal:
-            i = torch.arange(w.N_Q, device=dev)[:, None]
-            j = torch.arange(w.N_K, device=dev)[None, :]
-            mask = j > i + (w.N_K - w.N_Q)
-
-        def step():
-            for t in x:
-                t.grad = None
-            st = torch.matmul(x[0], x[1].transpose(-1, -2)).float() * w.scale_t
-            ss = torch.matmul(x[2], x[3].transpose(-1, -2)).float() * w.scale_s
-            if mask is not None:                  # finite fill: P = 0 there, and no inf - inf
-                st = st.masked_fill(mask, -1e9)
-                ss = ss.masked_fill(mask, -1e9)
-            logp, logq = F.log_softmax(st, -1), F.log_softmax(ss, -1)
-            kl = F.kl_div(logq, logp, reduction="none", log_target=True).sum(-1)
-            loss = kl.mean()
-            loss.backward()
-            return loss
-
+        mask = materialised_mask(w, dev)
         for _ in range(args.warmup):
-            step()
+            materialised_step(x, w, mask)
         torch.cuda.synchronize(dev)
         torch.cuda.reset_peak_memory_stats(dev)
         steps = min(args.steps, 20)
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record()
         for _ in range(steps):
-            step()
+            materialised_step(x, w, mask)
         t1.record()
         torch.cuda.synchronize(dev)
         ms = t0.elapsed_time(t1) / steps
@@ -352,6 +398,7 @@ def run_materialised(args, w):
         return 0
     line = dict(base, value=step_flops(w) / (ms * 1e-3) / 1e12, ms_per_step=ms, steps=steps,
                 warmup=args.warmup, higher_is_better=True,
+                dtype=f"bf16 inputs, logits by {_LOGITS_MODE.get(dev)}, fp32 softmax/KL",
                 peak_device_bytes=int(torch.cuda.max_memory_allocated(dev)))
     print(json.dumps(line), flush=True)
     return 0
@@ -420,7 +467,10 @@ def main():
 
     names = ["streamkl_fwd_kernel", "streamkl_mean_kernel", "streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"]
 
-    def step(ev=None, x=x):
+    outs0 = (kl, lt, ls, loss, dqs, dks, dqt, dkt)
+
+    def step(ev=None, x=x, o=outs0):
+        kl, lt, ls, loss, dqs, dks, dqt, dkt = o
         if flush is not None:
             flush.zero_()
         if ev is not None:
@@ -503,59 +553,89 @@ def main():
     code = skl.streamkl_check(stream)
 
     # End to end through the public API: every step copies its inputs from pinned
-    # host memory to the device and reads the loss back.  The copies run on a
-    # second stream into one of two device input sets, so step k+1's upload
-    # overlaps step k's kernels (both inside the timed region).
-    loss_h = torch.empty((), dtype=torch.float32).pin_memory()
+    # host memory to the device and reads its results back to pinned host memory
+    # (the loss and all gradients; the per-row KL and LSEs stay on the device as
+    # the backward's inputs).  Uploads run on one copy stream into one of two
+    # device input sets, downloads on another from one of two device output sets,
+    # so step k+1's upload and step k-1's download overlap step k's kernels (all
+    # inside the timed region).  A second variant reads back only the loss.
     h2d = sum(t.numel() * t.element_size() for t in host)
     xs = [x, [torch.empty_like(t) for t in x]]
-    copy_stream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event() for _ in range(2)]
-    used = [torch.cuda.Event() for _ in range(2)]
+    outs = [outs0, tuple(None if t is None else torch.empty_like(t) for t in outs0)]
+    back = [(3, 4, 5, 6, 7), (3,)]                   # output indices read back: everything / the loss only
+    host_out = [None if t is None else torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs0]
+    up_stream, down_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in range(2)]  # inputs of set i uploaded
+    used = [torch.cuda.Event() for _ in range(2)]    # the step on set i is done
+    fetched = [torch.cuda.Event() for _ in range(2)] # outputs of set i downloaded
+    for e in fetched:
+        e.record(down_stream)
 
     def upload(i):
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(used[i])          # the step that last read set i is done
+        with torch.cuda.stream(up_stream):
+            up_stream.wait_event(used[i])            # the step that last read set i is done
             for dst, src in zip(xs[i], host):
                 dst.copy_(src, non_blocking=True)
-            copied[i].record(copy_stream)
+            copied[i].record(up_stream)
 
-    def e2e_run(n, start=None):
+    def download(i, which):
+        with torch.cuda.stream(down_stream):
+            down_stream.wait_event(used[i])
+            for j in back[which]:
+                if outs[i][j] is not None:
+                    host_out[j].copy_(outs[i][j], non_blocking=True)
+            fetched[i].record(down_stream)
+
+    def d2h_bytes(which):
+        return sum(outs0[j].numel() * outs0[j].element_size() for j in back[which] if outs0[j] is not None)
+
+    def e2e_run(n, which, start=None):
         if start is not None:
-            copy_stream.wait_event(start)
+            up_stream.wait_event(start)
+            down_stream.wait_event(start)
         upload(0)
         for k in range(n):
             cur = k & 1
             if k + 1 < n:
                 upload(cur ^ 1)
             stream.wait_event(copied[cur])
-            step(x=xs[cur])
+            stream.wait_event(fetched[cur])          # set cur's previous results are on the host
+            step(x=xs[cur], o=outs[cur])
             used[cur].record(stream)
-            loss_h.copy_(loss, non_blocking=True)
+            download(cur, which)
+        stream.wait_event(fetched[(n - 1) & 1])      # the last results are on the host
 
-    e2e_run(args.warmup)
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    e2e_run(K, start=e0)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms_e2e = e0.elapsed_time(e1)
+    ms_e2e = []
+    for which in range(2):
+        e2e_run(args.warmup, which)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        e2e_run(K, which, start=e0)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e.append(e0.elapsed_time(e1))
+    ms_e2e, ms_e2e_loss = ms_e2e
 
     if world > 1:
-        ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], world, dev)
+        ms_total, ms_e2e, ms_e2e_loss = max_over_ranks([ms_total, ms_e2e, ms_e2e_loss], world, dev)
 
     ms_step = ms_total / K
     flops = step_flops(w)
     value = job_throughput(flops, world, ms_step)
     e2e_value = job_throughput(flops, world, ms_e2e / K)
+    e2e_loss_value = job_throughput(flops, world, ms_e2e_loss / K)
 
     sustained, burst, peak_src = measured_peak()
-    kf = kernel_flops(w)
+    kf, km = kernel_flops(w), kernel_method_flops(w)
     dominant = max((n for n in names if kf[n] > 0), key=lambda n: per_kernel[n])
-    achieved = kf[dominant] / (per_kernel[dominant] * 1e-3) / 1e12
+    # the kernels are timed with CUDA events over millisecond launches, so the
+    # burst GEMM rate is the denominator; `achieved` counts the method's own
+    # FLOPs in the launch, `achieved_issued` every MMA FLOP it issues
+    achieved = km[dominant] / (per_kernel[dominant] * 1e-3) / 1e12
+    achieved_issued = kf[dominant] / (per_kernel[dominant] * 1e-3) / 1e12
     traffic = recorded_traffic(dominant, w.name)
 
     if rank == 0:
@@ -574,10 +654,12 @@ def main():
             "config": dict(workload_config(w), parallelism=f"independent problem per GPU x{world}"),
             "pct_of_nominal_bf16_peak": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
             "pct_of_measured_bf16_peak": 100.0 * value / world / burst,
-            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": sustained,
-                         "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
-                         "peak_source": f"bf16_tflops_sustained of {peak_src}",
-                         "flops_per_launch": kf[dominant]},
+            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": burst,
+                         "unit": "TFLOP/s", "frac": achieved / burst, "traffic": traffic,
+                         "frac_method": achieved / burst, "frac_issued": achieved_issued / burst,
+                         "achieved_issued": achieved_issued,
+                         "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                         "flops_per_launch": km[dominant], "issued_flops_per_launch": kf[dominant]},
             "kernels": {n: {"ms": per_kernel[n], "share": per_kernel[n] / total_k,
                             "mma_tflops": (kf[n] / (per_kernel[n] * 1e-3) / 1e12) if kf[n] else None}
                         for n in names},
@@ -586,7 +668,11 @@ def main():
                        "bwd_tflops": (flops - fwd_flops(w)) / (bwd_ms * 1e-3) / 1e12},
             "cublas_bf16_gemm_tflops_same_run": cublas_tflops,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h_bytes(0),
+                    "reads_back": "loss and every gradient (dQ_s, dK_s" + (", dQ_t, dK_t)" if w.teacher_grads else ")")},
+            "e2e_loss_only": {"value": e2e_loss_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                              "d2h_bytes_per_step": d2h_bytes(1)},
             "gpu_launches": launches_per_step * K,
             "memory": memory,
             "clocks": sampler.summary(),

@@ -63,3 +63,19 @@ def test_step_flops_follow_the_metric():
     assert not c.causal and not c.teacher_grads
     pairs = c.B * c.H * c.N_Q * c.N_K
     assert bench.step_flops(c) == (2 * 2 * (c.d_t + c.d_s) + 2 * 2 * c.d_s) * pairs
+
+
+def test_kernel_method_flops_split_the_step():
+    # the method's FLOPs of the step are the forward's logits plus, for each of
+    # the two backward kernels, its own contraction and half of the recompute;
+    # each backward kernel issues one whole recompute, i.e. a quarter more at d = 128
+    for name in ("causal_8k_d128", "cross_1k_64k", "causal_2k_d64"):
+        w = inputs.WORKLOADS[name]
+        km, kf = bench.kernel_method_flops(w), bench.kernel_flops(w)
+        assert abs(sum(km.values()) - bench.step_flops(w)) <= 1e-9 * bench.step_flops(w)
+        assert km["streamkl_fwd_kernel"] == kf["streamkl_fwd_kernel"]
+        pairs = bench.visible_pairs(w) * w.B * w.H
+        for k in ("streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"):
+            assert kf[k] - km[k] == (w.d_t + w.d_s) * pairs
+    w = inputs.WORKLOADS["causal_8k_d128"]
+    assert bench.kernel_method_flops(w)["streamkl_bwd_dkv_kernel"] == 3 * 256 * bench.visible_pairs(w) * w.H

@@ -129,15 +129,19 @@ def _dk_head_sums_vanish(dk, what):
     assert float((s.abs() / (ref + 1e-30)).max()) < 2e-3, what
 
 
-@pytest.mark.parametrize("name,head_sample", [("causal_8k_d128", 1), ("cross_1k_64k", 1),
-                                              ("causal_32k_d128", 0)])
+# Sampling of the large workloads: whole heads (every element of dQ and dK of
+# the head) where the oracle finishes them in seconds, 2 for the 8k and the
+# cross-attention workloads and 1 for the 32k one, plus 256 seeded rows
+# across all heads for dQ.
+@pytest.mark.parametrize("name,head_sample", [("causal_8k_d128", 2), ("cross_1k_64k", 2),
+                                              ("causal_32k_d128", 1)])
 def test_bwd_large_workload_sampled(name, head_sample):
     w = inputs.WORKLOADS[name]
     qt, kt, qs, ks = inputs.make_inputs(w)
     teacher = w.teacher_grads
     dqs, dks, dqt, dkt = gpu_grads(w, cuda(qt, kt, qs, ks), teacher)
     g = 1.0 / w.rows
-    rows = inputs.sample_rows(w, 24).numpy()
+    rows = inputs.sample_rows(w, 256).numpy()
     ref = oracle.sampled_rows(w, rows, g=g, teacher=teacher)
     assert_grad(to_np(dqs).reshape(-1, w.d_s)[rows], ref["dq_s"], name + " dq_s rows")
     if teacher:
@@ -153,6 +157,34 @@ def test_bwd_large_workload_sampled(name, head_sample):
         if teacher:
             assert_grad(to_np(dkt[b, h]), r[3][0, 0], f"{name} dk_t head {b},{h}")
             assert_grad(to_np(dqt[b, h]), r[2][0, 0], f"{name} dq_t head {b},{h}")
+
+
+@pytest.mark.parametrize("causal,per_row_g", [(True, False), (False, True)])
+def test_bwd_d128_student_only_many_items_per_cta(causal, per_row_g):
+    # d_t = d_s = 128 with student gradients only: the K rows live in tensor
+    # memory, so the persistent key-owner kernel runs (without the staged K
+    # rows: five Q stages do not fit beside them at d = 128).  2 x 8 heads x 32
+    # key tiles = 512 items for 148 SMs, so every CTA takes several items and
+    # its counters, ring and barrier phases cross item boundaries; every element
+    # of dK_s and dQ_s is compared with the oracle.
+    B, H, N, d = 2, 8, 4096, 128
+    w = inputs.custom(B=B, H=H, N_Q=N, N_K=N, d_t=d, d_s=d, causal=causal, student="noise", noise_std=0.5,
+                      seed=5151 + int(causal))
+    qt, kt, qs, ks = inputs.make_inputs(w)
+    if per_row_g:
+        g = torch.randn(B, H, N, generator=torch.Generator().manual_seed(78)) / (B * H * N)
+        dkl, dloss, g_ref = g.cuda(), 0.0, g.double().numpy()
+    else:
+        dkl, dloss, g_ref = None, 1.0, 1.0 / (B * H * N)
+    dqs, dks, dqt, dkt = gpu_grads(w, cuda(qt, kt, qs, ks), False, dkl, dloss)
+    assert dqt is None and dkt is None
+    r = oracle.bwd(qt, kt, qs, ks, w.scale_t, w.scale_s, causal, g=g_ref, teacher=False)
+    assert_grad(to_np(dks), r[1], "dk_s")
+    assert_grad(to_np(dqs), r[0], "dq_s")
+    # and per head, so that one wrong head cannot hide in the whole-tensor norm
+    for b in range(B):
+        for h in range(H):
+            assert_grad(to_np(dks[b, h]), r[1][b, h], f"dk_s head {b},{h}")
 
 
 def test_no_quadratic_device_memory():

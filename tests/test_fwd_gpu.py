@@ -75,19 +75,27 @@ def test_fwd_causal_2k_workload():
     run_and_compare(inputs.WORKLOADS["causal_2k_d64"])
 
 
-@pytest.mark.parametrize("name", ["causal_8k_d128", "causal_32k_d128", "cross_1k_64k"])
-def test_fwd_large_workload_sampled_rows(name):
+# Sampling of the large workloads: every row of 2 whole heads (8k, cross) or 1
+# (32k), plus 256 seeded rows across all heads and the first and last rows.
+@pytest.mark.parametrize("name,head_sample", [("causal_8k_d128", 2), ("causal_32k_d128", 1), ("cross_1k_64k", 2)])
+def test_fwd_large_workload_sampled_rows(name, head_sample):
     w = inputs.WORKLOADS[name]
     qt, kt, qs, ks = inputs.make_inputs(w)
     kl, lt, ls, loss = streamkl_fwd(*cuda(qt, kt, qs, ks), w.scale_t, w.scale_s, w.causal)
     assert streamkl_check() == 0
-    rows = inputs.sample_rows(w, 48).numpy()
+    rows = inputs.sample_rows(w, 256).numpy()
     # include the first and last row of the first head and of the last head
     rows = np.unique(np.concatenate([rows, [0, w.N_Q - 1, w.rows - w.N_Q, w.rows - 1]]))
     ref = oracle.sampled_rows(w, rows)
     assert_kl(to_np(kl).ravel()[rows], ref["kl"], name)
     assert_lse(to_np(lt).ravel()[rows], ref["lse_t"], name + " lse_t")
     assert_lse(to_np(ls).ravel()[rows], ref["lse_s"], name + " lse_s")
+    for (b, h) in inputs.sample_heads(w, head_sample):
+        hq = [x[None, None] for x in inputs.head_inputs(w, b, h)]
+        rkl, rlt, rls = oracle.fwd(*hq, w.scale_t, w.scale_s, w.causal)
+        assert_kl(to_np(kl[b, h]), rkl, f"{name} head {b},{h}")
+        assert_lse(to_np(lt[b, h]), rlt, f"{name} head {b},{h} lse_t")
+        assert_lse(to_np(ls[b, h]), rls, f"{name} head {b},{h} lse_s")
     k = to_np(kl)
     assert np.isfinite(k).all() and k.min() > -1e-3
     assert abs(float(loss) - k.mean()) <= 1e-5 * max(1.0, abs(k.mean()))
