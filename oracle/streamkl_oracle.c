@@ -28,7 +28,20 @@
  *   dQ_s[i] = scale_s * sum_j dS_s[j] K_s[j],  dK_s[j] += scale_s * dS_s[j] Q_s[i]
  *   and the same for the teacher with scale_t.
  *
- * Layouts: row-major [B, H, N, d] doubles; per-row outputs [B, H, N_Q].
+ * Two variants of the visible set and of the key heads (readings of the
+ * abstract's use cases, sparse-attention training and long-context
+ * distillation, which need padded batches and grouped key heads; the pages
+ * give no formula for either, so these are the plain readings):
+ *  - padding: with per-batch key lengths kv_len[b] (NULL = all N_K keys), key
+ *    j is visible to row i iff it is visible under the mask above AND
+ *    j < kv_len[b] (lengths outside [0, N_K] are clamped to it).  A row with no
+ *    visible key has KL = 0, LSE = -inf and no gradient (the empty sums).
+ *  - grouped key heads: K_t has H_kt heads and K_s has H_ks heads, each
+ *    dividing H; query head h of batch b reads key head h / (H / H_k) of the
+ *    same batch, and a key head's gradient is the sum over its query heads.
+ *
+ * Layouts: row-major [B, H, N_Q, d] queries and [B, H_k, N_K, d] keys in
+ * doubles; per-row outputs [B, H, N_Q].
  * Threads split the query rows; each thread keeps private dK accumulators that
  * are summed in thread order at the end (so a fixed thread count gives a fixed
  * result).  Return value 0 = ok, nonzero = bad arguments / out of memory.
@@ -43,13 +56,15 @@
 typedef struct {
     const double *q_t, *k_t, *q_s, *k_s;
     int B, H, N_Q, N_K, d_t, d_s, causal;
+    int H_kt, H_ks;                   /* key heads of the teacher / student */
+    const int *kv_len;                /* per-batch key lengths, or NULL */
     double scale_t, scale_s;
     /* forward outputs (may be NULL) */
     double *kl, *lse_t, *lse_s;
     /* backward: per-row upstream gradient (NULL = forward only) */
     const double *g;
     double *dq_s, *dq_t;              /* indexed like the inputs */
-    double *dk_s_priv, *dk_t_priv;    /* this thread's private [B,H,N_K,d] */
+    double *dk_s_priv, *dk_t_priv;    /* this thread's private [B,H_k,N_K,d] */
     /* the rows this worker owns: flat ids r = (b*H + h)*N_Q + i */
     const int64_t *rows;              /* NULL = contiguous range */
     int64_t r_begin, r_end;
@@ -62,6 +77,19 @@ static int num_visible(int i, int N_Q, int N_K, int causal)
     int n = last + 1;
     if (n < 0) n = 0;
     if (n > N_K) n = N_K;
+    return n;
+}
+
+/* Visible keys of row i of batch b: a prefix [0, n) of the keys. */
+static int row_visible(const work_t *w, int b, int i)
+{
+    int n = num_visible(i, w->N_Q, w->N_K, w->causal);
+    if (w->kv_len) {
+        int len = w->kv_len[b];
+        if (len < 0) len = 0;
+        if (len > w->N_K) len = w->N_K;
+        if (len < n) n = len;
+    }
     return n;
 }
 
@@ -88,11 +116,15 @@ static void one_row(const work_t *w, int64_t r, double *s_t, double *s_s)
     const int N_Q = w->N_Q, N_K = w->N_K, d_t = w->d_t, d_s = w->d_s;
     const int64_t bh = r / N_Q;
     const int i = (int)(r % N_Q);
+    const int b = (int)(bh / w->H), h = (int)(bh % w->H);
+    /* the key heads this query head reads */
+    const int64_t kht = (int64_t)b * w->H_kt + h / (w->H / w->H_kt);
+    const int64_t khs = (int64_t)b * w->H_ks + h / (w->H / w->H_ks);
     const double *qt = w->q_t + (bh * N_Q + i) * d_t;
     const double *qs = w->q_s + (bh * N_Q + i) * d_s;
-    const double *kt = w->k_t + bh * (int64_t)N_K * d_t;
-    const double *ks = w->k_s + bh * (int64_t)N_K * d_s;
-    const int n = num_visible(i, N_Q, N_K, w->causal);
+    const double *kt = w->k_t + kht * (int64_t)N_K * d_t;
+    const double *ks = w->k_s + khs * (int64_t)N_K * d_s;
+    const int n = row_visible(w, b, i);
 
     for (int j = 0; j < n; ++j) {
         s_t[j] = w->scale_t * dot(qt, kt + (int64_t)j * d_t, d_t);
@@ -115,8 +147,8 @@ static void one_row(const work_t *w, int64_t r, double *s_t, double *s_s)
     double *dqt = w->dq_t ? w->dq_t + (bh * N_Q + i) * d_t : NULL;
     if (dqs) memset(dqs, 0, sizeof(double) * d_s);
     if (dqt) memset(dqt, 0, sizeof(double) * d_t);
-    double *dks = w->dk_s_priv ? w->dk_s_priv + bh * (int64_t)N_K * d_s : NULL;
-    double *dkt = w->dk_t_priv ? w->dk_t_priv + bh * (int64_t)N_K * d_t : NULL;
+    double *dks = w->dk_s_priv ? w->dk_s_priv + khs * (int64_t)N_K * d_s : NULL;
+    double *dkt = w->dk_t_priv ? w->dk_t_priv + kht * (int64_t)N_K * d_t : NULL;
     for (int j = 0; j < n; ++j) {
         const double logp = s_t[j] - lse_t, logq = s_s[j] - lse_s;
         const double p = exp(logp), q = exp(logq);
@@ -153,9 +185,10 @@ static int pick_threads(int nthreads, int64_t nrows)
     return nthreads;
 }
 
-static int check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal)
+static int check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal, int H_kt, int H_ks)
 {
     if (B < 0 || H < 0 || N_Q < 0 || N_K < 0 || d_t <= 0 || d_s <= 0) return 1;
+    if (H_kt <= 0 || H_ks <= 0 || (H > 0 && (H % H_kt || H % H_ks))) return 1;
     if (causal && N_Q > N_K) return 1;     /* would leave rows with no visible key */
     if (!causal && N_K == 0 && N_Q > 0) return 1;
     return 0;
@@ -166,8 +199,8 @@ static int check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, int cau
 static int run(work_t proto, int64_t nrows, int nthreads, double *dk_s, double *dk_t)
 {
     const int T = pick_threads(nthreads, nrows);
-    const int64_t nk_s = (int64_t)proto.B * proto.H * proto.N_K * proto.d_s;
-    const int64_t nk_t = (int64_t)proto.B * proto.H * proto.N_K * proto.d_t;
+    const int64_t nk_s = (int64_t)proto.B * proto.H_ks * proto.N_K * proto.d_s;
+    const int64_t nk_t = (int64_t)proto.B * proto.H_kt * proto.N_K * proto.d_t;
     work_t *ws = (work_t *)calloc((size_t)T, sizeof(work_t));
     pthread_t *th = (pthread_t *)calloc((size_t)T, sizeof(pthread_t));
     if (!ws || !th) { free(ws); free(th); return 2; }
@@ -194,17 +227,20 @@ static int run(work_t proto, int64_t nrows, int nthreads, double *dk_s, double *
     return err;
 }
 
-/* Forward: per-row KL and both log-sum-exps. */
+/* Forward: per-row KL and both log-sum-exps.  K_t, K_s have H_kt, H_ks
+ * heads; kv_len (per batch, nullable) hides padding keys. */
 int streamkl_oracle_fwd(const double *q_t, const double *k_t, const double *q_s, const double *k_s,
                         int B, int H, int N_Q, int N_K, int d_t, int d_s,
                         double scale_t, double scale_s, int causal,
+                        int H_kt, int H_ks, const int *kv_len,
                         double *kl, double *lse_t, double *lse_s, int nthreads)
 {
-    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal)) return 1;
+    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal, H_kt, H_ks)) return 1;
     work_t w;
     memset(&w, 0, sizeof w);
     w.q_t = q_t; w.k_t = k_t; w.q_s = q_s; w.k_s = k_s;
     w.B = B; w.H = H; w.N_Q = N_Q; w.N_K = N_K; w.d_t = d_t; w.d_s = d_s; w.causal = causal;
+    w.H_kt = H_kt; w.H_ks = H_ks; w.kv_len = kv_len;
     w.scale_t = scale_t; w.scale_s = scale_s;
     w.kl = kl; w.lse_t = lse_t; w.lse_s = lse_s;
     return run(w, (int64_t)B * H * N_Q, nthreads, NULL, NULL);
@@ -215,14 +251,16 @@ int streamkl_oracle_fwd(const double *q_t, const double *k_t, const double *q_s,
  * are recomputed here, from the inputs alone. */
 int streamkl_oracle_bwd(const double *q_t, const double *k_t, const double *q_s, const double *k_s,
                         int B, int H, int N_Q, int N_K, int d_t, int d_s,
-                        double scale_t, double scale_s, int causal, const double *g,
+                        double scale_t, double scale_s, int causal,
+                        int H_kt, int H_ks, const int *kv_len, const double *g,
                         double *dq_s, double *dk_s, double *dq_t, double *dk_t, int nthreads)
 {
-    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal) || !g) return 1;
+    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal, H_kt, H_ks) || !g) return 1;
     work_t w;
     memset(&w, 0, sizeof w);
     w.q_t = q_t; w.k_t = k_t; w.q_s = q_s; w.k_s = k_s;
     w.B = B; w.H = H; w.N_Q = N_Q; w.N_K = N_K; w.d_t = d_t; w.d_s = d_s; w.causal = causal;
+    w.H_kt = H_kt; w.H_ks = H_ks; w.kv_len = kv_len;
     w.scale_t = scale_t; w.scale_s = scale_s;
     w.g = g; w.dq_s = dq_s; w.dq_t = dq_t;
     return run(w, (int64_t)B * H * N_Q, nthreads, dk_s, dk_t);
@@ -234,17 +272,19 @@ int streamkl_oracle_bwd(const double *q_t, const double *k_t, const double *q_s,
 int streamkl_oracle_rows(const double *q_t, const double *k_t, const double *q_s, const double *k_s,
                          int B, int H, int N_Q, int N_K, int d_t, int d_s,
                          double scale_t, double scale_s, int causal,
+                        int H_kt, int H_ks, const int *kv_len,
                          const int64_t *rows, int64_t n_rows, const double *g,
                          double *kl, double *lse_t, double *lse_s,
                          double *dq_s, double *dq_t, int nthreads)
 {
-    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal)) return 1;
+    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal, H_kt, H_ks)) return 1;
     for (int64_t k = 0; k < n_rows; ++k)
         if (rows[k] < 0 || rows[k] >= (int64_t)B * H * N_Q) return 1;
     work_t w;
     memset(&w, 0, sizeof w);
     w.q_t = q_t; w.k_t = k_t; w.q_s = q_s; w.k_s = k_s;
     w.B = B; w.H = H; w.N_Q = N_Q; w.N_K = N_K; w.d_t = d_t; w.d_s = d_s; w.causal = causal;
+    w.H_kt = H_kt; w.H_ks = H_ks; w.kv_len = kv_len;
     w.scale_t = scale_t; w.scale_s = scale_s;
     w.kl = kl; w.lse_t = lse_t; w.lse_s = lse_s;
     w.g = g; w.dq_s = dq_s; w.dq_t = dq_t;
@@ -257,17 +297,19 @@ int streamkl_oracle_rows(const double *q_t, const double *k_t, const double *q_s
  * time the oracle on a bounded sample of a large problem. */
 int streamkl_oracle_bwd_rows(const double *q_t, const double *k_t, const double *q_s, const double *k_s,
                              int B, int H, int N_Q, int N_K, int d_t, int d_s,
-                             double scale_t, double scale_s, int causal, const double *g,
+                             double scale_t, double scale_s, int causal,
+                        int H_kt, int H_ks, const int *kv_len, const double *g,
                              const int64_t *rows, int64_t n_rows,
                              double *dq_s, double *dk_s, double *dq_t, double *dk_t, int nthreads)
 {
-    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal) || !g) return 1;
+    if (check_shape(B, H, N_Q, N_K, d_t, d_s, causal, H_kt, H_ks) || !g) return 1;
     for (int64_t k = 0; k < n_rows; ++k)
         if (rows[k] < 0 || rows[k] >= (int64_t)B * H * N_Q) return 1;
     work_t w;
     memset(&w, 0, sizeof w);
     w.q_t = q_t; w.k_t = k_t; w.q_s = q_s; w.k_s = k_s;
     w.B = B; w.H = H; w.N_Q = N_Q; w.N_K = N_K; w.d_t = d_t; w.d_s = d_s; w.causal = causal;
+    w.H_kt = H_kt; w.H_ks = H_ks; w.kv_len = kv_len;
     w.scale_t = scale_t; w.scale_s = scale_s;
     w.g = g; w.dq_s = dq_s; w.dq_t = dq_t;
     w.rows = rows;
