@@ -42,10 +42,11 @@ class StreamKLFunction(torch.autograd.Function):
     """loss = t2 * reduce(KL rows); see ``streamkl_loss`` for the arguments."""
 
     @staticmethod
-    def forward(ctx, q_t, k_t, q_s, k_s, scale_t, scale_s, causal, t2, reduction):
-        kl, lse_t, lse_s, _ = streamkl_fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, loss_mean=False)
+    def forward(ctx, q_t, k_t, q_s, k_s, scale_t, scale_s, causal, t2, reduction, kv_len):
+        kl, lse_t, lse_s, _ = streamkl_fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, loss_mean=False,
+                                           kv_len=kv_len)
         ctx.save_for_backward(q_t, k_t, q_s, k_s, kl, lse_t, lse_s)
-        ctx.cfg = (scale_t, scale_s, causal, t2, reduction)
+        ctx.cfg = (scale_t, scale_s, causal, t2, reduction, kv_len)
         ctx.mark_non_differentiable(lse_t, lse_s)
         n = kl.numel()
         if reduction == "mean":
@@ -59,25 +60,25 @@ class StreamKLFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, grad_out, _g_lse_t, _g_lse_s):
         q_t, k_t, q_s, k_s, kl, lse_t, lse_s = ctx.saved_tensors
-        scale_t, scale_s, causal, t2, reduction = ctx.cfg
+        scale_t, scale_s, causal, t2, reduction, kv_len = ctx.cfg
         teacher = ctx.needs_input_grad[0] or ctx.needs_input_grad[1]
         if grad_out is None:
-            return (None,) * 9
+            return (None,) * 10
         if reduction == "none":
             dkl = grad_out.float().contiguous()
             dq_s, dk_s, dq_t, dk_t = streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s, causal,
-                                                  dkl=dkl, teacher_grads=teacher)
+                                                  dkl=dkl, teacher_grads=teacher, kv_len=kv_len)
         else:
             g = grad_out.float().reshape(1)
             n = kl.numel()
             scale = t2 / n if reduction == "mean" else t2
             dq_s, dk_s, dq_t, dk_t = streamkl_bwd(q_t, k_t, q_s, k_s, kl, lse_t, lse_s, scale_t, scale_s, causal,
-                                                  dloss=g, dloss_scale=scale, teacher_grads=teacher)
-        return dq_t, dk_t, dq_s, dk_s, None, None, None, None, None
+                                                  dloss=g, dloss_scale=scale, teacher_grads=teacher, kv_len=kv_len)
+        return dq_t, dk_t, dq_s, dk_s, None, None, None, None, None, None
 
 
 def streamkl_loss(q_t, k_t, q_s, k_s, *, causal=False, temperature=1.0, scale_t=None, scale_s=None,
-                  reduction="mean", return_lse=False):
+                  reduction="mean", return_lse=False, kv_len=None):
     """Distillation loss between the teacher's and the student's attention.
 
     q_t, k_t: teacher queries/keys [B, H, N_Q|N_K, d_t]; q_s, k_s: the
@@ -88,10 +89,14 @@ def streamkl_loss(q_t, k_t, q_s, k_s, *, causal=False, temperature=1.0, scale_t=
     "none" (the per-row KL of the softened distributions, [B, H, N_Q],
     without the T^2 factor: multiply by T^2 before reducing it yourself).
     With return_lse the per-row log-sum-exps of both softened distributions
-    are returned too (no gradient).
+    are returned too (no gradient).  Keys may have fewer heads than the
+    queries (grouped key heads), and kv_len (int32 [B] on the device) marks
+    the keys at and past each batch element's length as padding; "mean" and
+    "sum" still run over every query row (reduce "none" with your own row
+    weights to leave padded query rows out).
     """
     if reduction not in _REDUCTIONS:
         raise ValueError(f"reduction must be one of {_REDUCTIONS}")
     st, ss, t2 = _scales(q_t.shape[-1], q_s.shape[-1], temperature, scale_t, scale_s)
-    out, lse_t, lse_s = StreamKLFunction.apply(q_t, k_t, q_s, k_s, st, ss, bool(causal), t2, reduction)
+    out, lse_t, lse_s = StreamKLFunction.apply(q_t, k_t, q_s, k_s, st, ss, bool(causal), t2, reduction, kv_len)
     return (out, lse_t, lse_s) if return_lse else out

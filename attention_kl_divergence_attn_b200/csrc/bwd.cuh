@@ -57,6 +57,8 @@ namespace skl {
 
 struct BwdParams {
     int BH, N_Q, N_K, causal, n_tiles;
+    int H, Hkt, Hks;              // query heads per batch element, key heads of K_t and K_s
+    const int *kv_len;            // per-batch key lengths (padding), or null
     int splits;                   // query-owner kernel: key ranges per query tile (1 = whole row)
     float ct, cs;                 // scale * log2(e)
     float out_t, out_s;           // output scales: scale_t * ln2 (teacher), scale_s (student)
@@ -265,7 +267,9 @@ constexpr int kBwdChunk = 64 / kBwdHalves;
 
 // Writes NCOLS (16 or 32) accumulator columns of this warp's 32 TMEM lanes
 // (rows row0 .. row0+31 of the output, of which the first nvalid exist) to
-// global memory, scaled by `scale` (per thread = per row).  Each thread first
+// global memory, scaled by `scale` (per thread = per row), or zeros for the
+// rows whose thread passes `zero` (a padding key, or no visible pair at all:
+// the accumulator is then not read as a value, so nothing in it can leak).  Each thread first
 // puts its row into a per-warp staging tile in shared memory with 16-byte
 // stores (row stride NCOLS + 4 floats: rows stay 16-byte aligned and the eight
 // rows written by a quarter-warp fall into different banks), then the warp
@@ -277,7 +281,7 @@ constexpr int kDrainPad = 4;
 
 template <int NCOLS>
 __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *dst, size_t ld, int nvalid,
-                                           float *stage, int lane) {
+                                           float *stage, int lane, bool zero) {
     static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
     constexpr int SP = NCOLS + kDrainPad, V = NCOLS / 4, RPI = 32 / V;
     float4 *mine = reinterpret_cast<float4 *>(stage + lane * SP);
@@ -288,8 +292,9 @@ __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *d
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mine[c / 4 + k] =
-                make_float4(v[4 * k] * scale, v[4 * k + 1] * scale, v[4 * k + 2] * scale, v[4 * k + 3] * scale);
+            mine[c / 4 + k] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                   : make_float4(v[4 * k] * scale, v[4 * k + 1] * scale, v[4 * k + 2] * scale,
+                                                 v[4 * k + 3] * scale);
     }
     __syncwarp();
     const int rr = lane / V, c4 = (lane % V) * 4;
@@ -304,11 +309,11 @@ __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *d
 }
 
 // Writes NCOLS (16 or 32) accumulator columns of this thread's TMEM lane,
-// scaled by `scale`, to its output row at `dst` (when `valid`), straight from
-// registers: 32-byte stores when `dst` is 32-byte aligned (whole sectors),
+// scaled by `scale` (or zeros when `zero`), to its output row at `dst` (when
+// `valid`), straight from registers: 32-byte stores when `dst` is 32-byte aligned (whole sectors),
 // else 16-byte stores.
 template <int NCOLS>
-__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool valid) {
+__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool valid, bool zero) {
     static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
     const bool a32 = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
 #pragma unroll
@@ -317,7 +322,7 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *ds
         tmem_ld16(taddr + c, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] *= scale;
+        for (int k = 0; k < 16; ++k) v[k] = zero ? 0.f : v[k] * scale;
         if (valid) {
             if (a32) {
                 st_global_v8(dst + c, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
@@ -382,7 +387,10 @@ struct DkvCfg {
     static constexpr uint32_t IDESC_KT = idesc_bf16(128, DT, 0, 1);
 };
 
-template <int DT, int DS, bool TEACHER>
+// PAD: the problem has per-batch key lengths (padding).  A separate
+// instantiation, because the padding checks cost registers that the tile loop
+// of the d = 128 teacher-and-student form, at the register limit, does not have.
+template <int DT, int DS, bool TEACHER, bool PAD>
 __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     streamkl_bwd_dkv_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
                             const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
@@ -409,6 +417,23 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     const int n_qt_all = (p.N_Q + C::BM - 1) / C::BM;
     const int first_qt = p.causal ? max(0, k0 - off) / C::BM : 0;
     const int n_qt = max(0, n_qt_all - first_qt);
+    const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);   // this head's key heads
+    if constexpr (PAD) {
+        // A CTA whose keys are all padding has no visible pair: it writes its
+        // zero dK rows and returns before any set-up (a whole-CTA decision, so
+        // no barrier, copy or tensor memory is involved yet).
+        const int nk = key_count(p.kv_len, bh / p.H, p.N_K, p.st.word, threadIdx.x == 0 && kt_idx == 0);
+        if (k0 >= nk) {
+            const int rows = min(C::BN, p.N_K - k0);
+            float4 *ds4 = reinterpret_cast<float4 *>(p.dk_s + ((size_t)bh * p.N_K + k0) * DS);
+            for (int e = threadIdx.x; e < rows * DS / 4; e += C::THREADS) ds4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (TEACHER) {
+                float4 *dt4 = reinterpret_cast<float4 *>(p.dk_t + ((size_t)bh * p.N_K + k0) * DT);
+                for (int e = threadIdx.x; e < rows * DT / 4; e += C::THREADS) dt4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            return;
+        }
+    }
 
     // Set-up.  Each warp has its own part, and the block barrier below waits
     // for the slowest: issuing a TMA copy takes a while, so before the barrier
@@ -433,9 +458,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 prefetch_tmap(&mKt); prefetch_tmap(&mKs);
                 mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
 #pragma unroll
-                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
             }
             prefetch_tmap(&mQt); prefetch_tmap(&mQs);
             if (n_qt > 0) {
@@ -478,8 +503,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     if constexpr (C::K_TMEM) {
         if (warp >= 2) {
             const int wg = (warp - 2) >> 2, sub = warp & 3;
-            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
-            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bkt, p.N_K, k0, wg, sub, lane);
+            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bks, p.N_K, k0, wg, sub, lane);
             tmem_st_wait();
         }
         tc_fence_before();
@@ -676,11 +701,14 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             const size_t r0 = (size_t)bh * p.N_K + row0;
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
             const float gs = p.dkl ? 1.f : g_uni;         // a uniform g was left out of dS
+            // a padding key: its row is zero (the length is read again here rather
+            // than kept live through the tile loop)
+            const bool pad = PAD && gk >= key_count(p.kv_len, bh / p.H, p.N_K, nullptr, false);
             drain_rows<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + r0 * DS + wg * HS, DS, nvalid,
-                           stage, lane);
+                           stage, lane, pad);
             if (TEACHER)
                 drain_rows<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + r0 * DT + wg * HT, DT,
-                               nvalid, stage, lane);
+                               nvalid, stage, lane, pad);
         } else if (n_qt == 0 && gk < p.N_K && wg == 0) {
             const size_t r = (size_t)bh * p.N_K + gk;
             for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
@@ -743,12 +771,14 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     const int off = p.N_K - p.N_Q;
     const int n_qt_all = (p.N_Q + C::BM - 1) / C::BM;
     const int n_items = p.BH * p.n_tiles;
-    // item j: key tile j / BH (low key tiles see the most queries), head j % BH
+    // item j: key tile j / BH (low key tiles see the most queries), head j % BH;
+    // an item whose keys are all padding has no visible pair (zero dK rows)
     auto item_geom = [&](int j, int &k0, int &bh, int &first_qt, int &n_qt) {
         k0 = (j / p.BH) * C::BN;
         bh = j % p.BH;
         first_qt = p.causal ? max(0, k0 - off) / C::BM : 0;
         n_qt = max(0, n_qt_all - first_qt);
+        if (p.kv_len && k0 >= key_count(p.kv_len, bh / p.H, p.N_K, nullptr, false)) n_qt = 0;
     };
 
     if (warp == 0) {
@@ -778,19 +808,20 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             int k0, bh, first_qt, n_qt;
             item_geom(persistent_item(0, n_items), k0, bh, first_qt, n_qt);
             if (n_qt > 0) {
+                const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);
                 if (!C::K_TMEM) {
                     mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
 #pragma unroll
-                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
                 } else if (C::K_STAGED) {
                     mbar_expect_tx(&bar_kst, C::KST_BYTES);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, k0, bh);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, k0, bkt);
 #pragma unroll
                     for (int b = 0; b < DS / 64; ++b)
-                        tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, k0, bh);
+                        tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, k0, bks);
                 }
                 mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
 #pragma unroll
@@ -861,12 +892,13 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 if (!mbar_wait(&bar_kstfree, (kst_n - 1) & 1, p.st, abort_v, 20)) return false;
             }
             mbar_expect_tx(&bar_kst, C::KST_BYTES);
+            const int kbt = key_head(kst_bh, p.H, p.Hkt), kbs = key_head(kst_bh, p.H, p.Hks);
 #pragma unroll
             for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kst_bh);
+                tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kbt);
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kst_bh);
+                tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kbs);
             ++kst_n;
             ++kst_r;
             kst_find();
@@ -893,10 +925,11 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 if (it > 0 && !mbar_wait(&bar_kfree, (it - 1) & 1, p.st, abort_v, 10)) break;
                 if (lane == 0) {
                     mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
+                    const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bh);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
 #pragma unroll
-                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bh);
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
                 }
             }
             if (!C::K_TMEM) ++k_issued;
@@ -908,9 +941,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     int k0n, bhn, fqn, nqn;
                     item_geom(jn, k0n, bhn, fqn, nqn);
                     const int rows = min(C::BN, p.N_K - k0n);
-                    const size_t base = (size_t)bhn * p.N_K + k0n;
-                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.kt_raw) + base * DT, (uint32_t)rows * DT * 2);
-                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.ks_raw) + base * DS, (uint32_t)rows * DS * 2);
+                    const size_t bt = (size_t)key_head(bhn, p.H, p.Hkt) * p.N_K + k0n;
+                    const size_t bs = (size_t)key_head(bhn, p.H, p.Hks) * p.N_K + k0n;
+                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.kt_raw) + bt * DT, (uint32_t)rows * DT * 2);
+                    prefetch_l2(static_cast<const __nv_bfloat16 *>(p.ks_raw) + bs * DS, (uint32_t)rows * DS * 2);
                 }
             }
             // Per-query constants of a tile: lane l handles queries l and l + 32.
@@ -1105,8 +1139,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 tile_rows_to_tmem<DS>(lane_base + C::TMEM_KS, sKst + C::BN * DT * 2, wg, row);
             } else {
                 tc_fence_after();
-                resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bh, p.N_K, k0, wg, sub, lane);
-                resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bh, p.N_K, k0, wg, sub, lane);
+                resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, key_head(bh, p.H, p.Hkt), p.N_K, k0, wg, sub, lane);
+                resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, key_head(bh, p.H, p.Hks), p.N_K, k0, wg, sub, lane);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -1183,11 +1217,14 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 // dK rows straight from tensor memory to global memory (the stage
                 // ring already holds the next item's tiles)
                 const bool valid = gk < p.N_K;
+                const bool pad = gk >= key_count(p.kv_len, bh / p.H, p.N_K, nullptr, false);   // zero row
                 const size_t grow = (size_t)bh * p.N_K + gk;
                 constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
-                drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + grow * DS + wg * HS, valid);
+                drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + grow * DS + wg * HS, valid,
+                              pad);
                 if (TEACHER)
-                    drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + grow * DT + wg * HT, valid);
+                    drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + grow * DT + wg * HT, valid,
+                                  pad);
                 tc_fence_before();
                 g0 += n_qt;
                 ++it;
@@ -1259,10 +1296,14 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     const int bh = (int)(blockIdx.x % p.BH);
     const int q0 = qt_idx * C::BM;
     const int off = p.N_K - p.N_Q;
-    int kend = p.N_K;
-    if (p.causal) kend = min(p.N_K, min(q0 + C::BM - 1, p.N_Q - 1) + off + 1);
+    // this head's key heads, and its keys that are not padding
+    const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);
+    const int nk = key_count(p.kv_len, bh / p.H, p.N_K, p.st.word, false);
+    int kend = nk;
+    if (p.causal) kend = min(nk, min(q0 + C::BM - 1, p.N_Q - 1) + off + 1);
     const int n_all = (kend + C::BN - 1) / C::BN;
-    // this CTA's key tiles [kt_lo, kt_lo + n_kt) (the host keeps n_kt >= 1); loops count from 0
+    // this CTA's key tiles [kt_lo, kt_lo + n_kt); loops count from 0.  With
+    // padding a range may be empty (n_kt = 0): the CTA then writes zeros.
     const int kt_lo = (int)((long long)n_all * split / p.splits);
     const int n_kt = (int)((long long)n_all * (split + 1) / p.splits) - kt_lo;
 
@@ -1293,12 +1334,15 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
         }
-        mbar_expect_tx(&bar_kfull[0], C::STAGE_BYTES);
+        if (n_kt > 0) {
+            mbar_expect_tx(&bar_kfull[0], C::STAGE_BYTES);
 #pragma unroll
-        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, kt_lo * C::BN, bh);
+            for (int b = 0; b < DT / 64; ++b)
+                tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, kt_lo * C::BN, bkt);
 #pragma unroll
-        for (int b = 0; b < DS / 64; ++b)
-            tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, kt_lo * C::BN, bh);
+            for (int b = 0; b < DS / 64; ++b)
+                tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, kt_lo * C::BN, bks);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -1333,11 +1377,11 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bh);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
-                                bh);
+                                bks);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -1436,7 +1480,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             g = p.dkl ? p.dkl[r] : uniform_g(p);
             KL2 = p.kl[r] * kLog2eF;
         }
-        const int lim = p.causal ? min(p.N_K, gq + off + 1) : p.N_K;   // first hidden key
+        const int lim = p.causal ? min(nk, gq + off + 1) : nk;   // first hidden key
         bool ok = true;
         for (int kt = par; kt < n_kt; kt += kBwdParities) {
             const int buf = kt & 1;
@@ -1444,7 +1488,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             tc_fence_after();
             const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
             const int kb = (kt_lo + kt) * C::BN + half * CW;
-            const bool masked = (kb + CW > p.N_K) || (p.causal && (kb + CW - 1 > q0 + off));
+            const bool masked = (kb + CW > nk) || (p.causal && (kb + CW - 1 > q0 + off));
             if (masked)
                 dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, &bar_ssfree[buf]);
             else
@@ -1468,12 +1512,12 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 dst_t = p.part_t;
             }
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
-            // the row's g was left out of dS
+            // the row's g was left out of dS; no key tile: nothing was accumulated
             drain_rows<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s * g, dst_s + r0 * DS + wg * HS, DS, nvalid,
-                           stage, lane);
+                           stage, lane, n_kt == 0);
             if (TEACHER)
                 drain_rows<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t * g, dst_t + r0 * DT + wg * HT, DT, nvalid,
-                               stage, lane);
+                               stage, lane, n_kt == 0);
         }
     }
 
@@ -1482,6 +1526,30 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// Grouped key heads: the key-owner kernel writes one dK partial per query head
+// ([B, H, N_K, d]); a key head's gradient is the sum of its group's partials,
+// out[b, g] = sum over u = 0 .. G-1 of part[b, g G + u], in that order
+// (deterministic).  nd = N_K * d, a multiple of 4; 16-byte aligned arrays.
+__global__ void __launch_bounds__(256) streamkl_group_sum_kernel(const float *__restrict__ part, int H, int Hk,
+                                                                 long long nd, long long n_out,
+                                                                 float *__restrict__ out) {
+    const int G = H / Hk;
+    const long long nd4 = nd >> 2;
+    const float4 *p4 = reinterpret_cast<const float4 *>(part);
+    float4 *o4 = reinterpret_cast<float4 *>(out);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (n_out >> 2);
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long bg = i / nd4, e = i - bg * nd4;          // key head b * Hk + g, element
+        const long long first = (bg / Hk) * H + (bg % Hk) * G;   // its group's first query head
+        float4 a = __ldg(p4 + first * nd4 + e);
+        for (int u = 1; u < G; ++u) {
+            const float4 b = __ldg(p4 + (first + u) * nd4 + e);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        o4[i] = a;
     }
 }
 

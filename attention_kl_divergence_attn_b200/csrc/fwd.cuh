@@ -42,6 +42,8 @@ namespace skl {
 
 struct FwdParams {
     int BH, N_Q, N_K, causal, n_qt;
+    int H, Hkt, Hks;       // query heads per batch element, key heads of K_t and K_s
+    const int *kv_len;     // per-batch key lengths (padding), or null
     int splits;            // key ranges per query tile (1 = the whole row in one CTA)
     float ct, cs;          // scale_t * log2(e), scale_s * log2(e)
     float *kl, *lse_t, *lse_s;
@@ -70,9 +72,16 @@ __device__ __forceinline__ void merge_state(RowState &a, const RowState &b) {
 }
 
 // Row outputs from a complete state: LSE = ln2 (M + log2 l) for each
-// distribution and KL = ln2 (A / l_t) - LSE_t + LSE_s.
+// distribution and KL = ln2 (A / l_t) - LSE_t + LSE_s.  A row that saw no key
+// (all keys padding) has the empty sums: KL = 0, LSE = -inf.
 __device__ __forceinline__ void finish_row(const RowState &x, float *kl, float *lse_t, float *lse_s) {
     const float LN2 = 0.69314718055994530942f;
+    if (x.lt == 0.f) {
+        *kl = 0.f;
+        *lse_t = -INFINITY;
+        *lse_s = -INFINITY;
+        return;
+    }
     const float lse_t2 = x.Mt + lg2(x.lt), lse_s2 = x.Ms + lg2(x.ls);
     *lse_t = lse_t2 * LN2;
     *lse_s = lse_s2 * LN2;
@@ -108,12 +117,14 @@ struct FwdCfg {
     static_assert(TMEM_QS + DS / 2 <= TMEM_COLS, "logit buffers and query rows fit tensor memory");
 };
 
-// Number of key tiles a 128-row query tile starting at q0 must visit.
-__device__ __forceinline__ int fwd_key_tiles(int q0, int N_Q, int N_K, int causal, int BN) {
-    int kend = N_K;
+// Number of key tiles a 128-row query tile starting at q0 must visit: keys
+// below nk (the keys that are not padding) and, under the causal mask, at or
+// below the tile's last row + off (off = N_K - N_Q).
+__device__ __forceinline__ int fwd_key_tiles(int q0, int N_Q, int nk, int off, int causal, int BN) {
+    int kend = nk;
     if (causal) {
         int last_row = min(q0 + 127, N_Q - 1);
-        kend = min(N_K, last_row + (N_K - N_Q) + 1);
+        kend = min(nk, last_row + off + 1);
     }
     return (kend + BN - 1) / BN;
 }
@@ -270,11 +281,15 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     const int qt_idx = p.n_qt - 1 - lin / p.splits;
     const int bh = (int)(blockIdx.x % p.BH);
     const int q0 = qt_idx * C::BM;
-    const int n_all = fwd_key_tiles(q0, p.N_Q, p.N_K, p.causal, C::BN);
+    const int off = p.N_K - p.N_Q;
+    // keys of this head: its key heads (grouped key heads) and its batch
+    // element's keys that are not padding
+    const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);
+    const int nk = key_count(p.kv_len, bh / p.H, p.N_K, p.st.word, threadIdx.x == 0 && split == 0);
+    const int n_all = fwd_key_tiles(q0, p.N_Q, nk, off, p.causal, C::BN);
     // this CTA's key tiles [kt_lo, kt_lo + n_kt); loops below count from 0
     const int kt_lo = (int)((long long)n_all * split / p.splits);
     const int n_kt = (int)((long long)n_all * (split + 1) / p.splits) - kt_lo;
-    const int off = p.N_K - p.N_Q;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar_q, 1);
@@ -304,10 +319,10 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
 #pragma unroll
             for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bkt);
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bh);
+                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bks);
         }
     }
     if (warp == 1) {
@@ -332,11 +347,11 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bh);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
-                                bh);
+                                bks);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -411,9 +426,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 tmem_ld32(bufc + c * 32, ut);
                 tmem_ld32(bufc + 64 + c * 32, us);
                 tmem_ld_wait();
-                const bool masked = (kc + 32 > p.N_K) || (p.causal && (kc + 31 > q0 + off));
+                const bool masked = (kc + 32 > nk) || (p.causal && (kc + 31 > q0 + off));
                 if (masked) {
-                    const int lim = p.causal ? min(p.N_K, grow + off + 1) : p.N_K;   // first hidden key
+                    const int lim = p.causal ? min(nk, grow + off + 1) : nk;   // first hidden key
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
                         if (kc + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }

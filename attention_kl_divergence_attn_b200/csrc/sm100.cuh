@@ -16,6 +16,7 @@ namespace skl {
 // Bit layout of the device status word that lives in the caller's workspace.
 enum : uint32_t {
     kStatusTimeout = 1u << 0,   // some bounded wait gave up
+    kStatusBadLength = 1u << 1, // a per-batch key length outside [0, N_K] (clamped)
     kStatusWhoShift = 8,        // bits 8..15: which wait (role-specific id)
 };
 
@@ -23,6 +24,21 @@ struct DevStatus {
     uint32_t *word;             // device status word (workspace)
     unsigned long long budget_ns;
 };
+
+// ---------------------------------------------------------------- problem geometry
+// Grouped key heads: query head bh = b * H + h reads key head
+// b * Hk + h / (H / Hk) of a key tensor with Hk heads per batch element.
+__device__ __forceinline__ int key_head(int bh, int H, int Hk) { return (bh / H) * Hk + (bh % H) / (H / Hk); }
+
+// Keys of batch element b that are not padding: kv_len[b] clamped to
+// [0, N_K] (all N_K without lengths).  With `report`, a length outside that
+// range sets kStatusBadLength in the status word.
+__device__ __forceinline__ int key_count(const int *kv_len, int b, int N_K, uint32_t *word, bool report) {
+    if (!kv_len) return N_K;
+    const int len = __ldg(kv_len + b);
+    if (report && (len < 0 || len > N_K) && word) atomicOr(word, (uint32_t)kStatusBadLength);
+    return len < 0 ? 0 : (len > N_K ? N_K : len);
+}
 
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;

@@ -80,6 +80,15 @@ streamkl_status check_shape(int B, int H, int N_Q, int N_K, int d_t, int d_s, in
     return STREAMKL_OK;
 }
 
+// Grouped key heads and padding: K_t, K_s have H_kt, H_ks heads, each at
+// least 1 and dividing H; the key lengths (if any) are 4-byte aligned ints.
+streamkl_status check_heads(int H, int H_kt, int H_ks, const int *kv_len) {
+    if (H_kt < 1 || H_ks < 1 || H_kt > (1 << 24) || H_ks > (1 << 24)) return STREAMKL_ERR_INVALID_ARG;
+    if (H > 0 && (H % H_kt != 0 || H % H_ks != 0)) return STREAMKL_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return STREAMKL_ERR_INVALID_ARG;
+    return STREAMKL_OK;
+}
+
 // Input and output pointers of the forward: required (and 16-byte aligned)
 // unless the problem has no rows.  Makes no CUDA call.
 streamkl_status fwd_check_pointers(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
@@ -174,17 +183,32 @@ streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const C
 // Which backward kernels a call launches.
 enum BwdParts { kPartDK = 1, kPartDQ = 2 };
 
+// Where the key-owner kernel's dK goes when key heads are grouped: it writes
+// one partial per query head to the workspace (p.dk_s / p.dk_t point there),
+// and a fixed-order group sum writes each key head's gradient to these.
+struct DkOut {
+    float *dk_s, *dk_t;
+};
+
+streamkl_status group_sum(const float *part, int H, int Hk, int BK, int N_K, int d, float *out, cudaStream_t s) {
+    const long long nd = (long long)N_K * d, n_out = (long long)BK * nd;
+    const long long blocks = std::min<long long>((n_out / 4 + 255) / 256, 8ll * std::max(1, sm_count()));
+    streamkl_group_sum_kernel<<<(unsigned)std::max(1ll, blocks), 256, 0, s>>>(part, H, Hk, nd, n_out, out);
+    return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+}
+
 template <int DT, int DS, bool TEACHER>
 streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int N_Q, int N_K,
-                           BwdParams p, int parts, cudaStream_t stream) {
+                           BwdParams p, int parts, DkOut out, cudaStream_t stream) {
     using CK = DkvCfg<DT, DS, TEACHER>;
     using CQ = DqCfg<DT, DS, TEACHER>;
     const int BH = p.BH;
+    const int BKt = BH / p.H * p.Hkt, BKs = BH / p.H * p.Hks;   // key heads of K_t, K_s
     CUtensorMap mqt, mkt, mqs, mks;
     if (parts & kPartDK) {
         // key-owner kernel: K boxes of 128 rows, Q boxes of 64 rows
-        if (!make_map(&mqt, q_t, DT, N_Q, BH, CK::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CK::BN) ||
-            !make_map(&mqs, q_s, DS, N_Q, BH, CK::BM) || !make_map(&mks, k_s, DS, N_K, BH, CK::BN))
+        if (!make_map(&mqt, q_t, DT, N_Q, BH, CK::BM) || !make_map(&mkt, k_t, DT, N_K, BKt, CK::BN) ||
+            !make_map(&mqs, q_s, DS, N_Q, BH, CK::BM) || !make_map(&mks, k_s, DS, N_K, BKs, CK::BN))
             return STREAMKL_ERR_CUDA;
         p.n_tiles = (N_K + CK::BN - 1) / CK::BN;
         const long long items = (long long)BH * p.n_tiles;
@@ -193,16 +217,25 @@ streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, co
         // the items, overlapping each item's start with the previous one's end)
         // is faster; at the register limit (teacher and student K in shared
         // memory) one CTA per item keeps the inner loop faster.
-        auto kdkv = CK::K_TMEM ? streamkl_bwd_dkv_persistent_kernel<DT, DS, TEACHER> : streamkl_bwd_dkv_kernel<DT, DS, TEACHER>;
+        auto kdkv = CK::K_TMEM ? streamkl_bwd_dkv_persistent_kernel<DT, DS, TEACHER>
+                    : (p.kv_len ? streamkl_bwd_dkv_kernel<DT, DS, TEACHER, true>
+                                : streamkl_bwd_dkv_kernel<DT, DS, TEACHER, false>);
         if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
         const long long grid = CK::K_TMEM ? std::min<long long>(items, std::max(1, sm_count())) : items;
         kdkv<<<(unsigned)grid, CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+        // grouped key heads: each key head's gradient is its group's partials summed in order
+        streamkl_status st = STREAMKL_OK;
+        if (out.dk_s != p.dk_s && (st = group_sum(p.dk_s, p.H, p.Hks, BKs, N_K, DS, out.dk_s, stream)) != STREAMKL_OK)
+            return st;
+        if (TEACHER && out.dk_t != p.dk_t &&
+            (st = group_sum(p.dk_t, p.H, p.Hkt, BKt, N_K, DT, out.dk_t, stream)) != STREAMKL_OK)
+            return st;
     }
     if (parts & kPartDQ) {
         // query-owner kernel: Q boxes of 128 rows, K boxes of 64 rows
-        if (!make_map(&mqt, q_t, DT, N_Q, BH, CQ::BM) || !make_map(&mkt, k_t, DT, N_K, BH, CQ::BN) ||
-            !make_map(&mqs, q_s, DS, N_Q, BH, CQ::BM) || !make_map(&mks, k_s, DS, N_K, BH, CQ::BN))
+        if (!make_map(&mqt, q_t, DT, N_Q, BH, CQ::BM) || !make_map(&mkt, k_t, DT, N_K, BKt, CQ::BN) ||
+            !make_map(&mqs, q_s, DS, N_Q, BH, CQ::BM) || !make_map(&mks, k_s, DS, N_K, BKs, CQ::BN))
             return STREAMKL_ERR_CUDA;
         auto kdq = streamkl_bwd_dq_kernel<DT, DS, TEACHER>;
         if (set_smem(kdq, CQ::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
@@ -227,28 +260,41 @@ streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, co
 
 template <bool TEACHER>
 streamkl_status dispatch_bwd(int d_t, int d_s, const void *q_t, const void *k_t, const void *q_s, const void *k_s,
-                             int N_Q, int N_K, const BwdParams &p, int parts, cudaStream_t s) {
-    if (d_t == 64 && d_s == 64) return launch_bwd<64, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
-    if (d_t == 128 && d_s == 128) return launch_bwd<128, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
-    if (d_t == 128 && d_s == 64) return launch_bwd<128, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
-    return launch_bwd<64, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+                             int N_Q, int N_K, const BwdParams &p, int parts, DkOut out, cudaStream_t s) {
+    if (d_t == 64 && d_s == 64) return launch_bwd<64, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s);
+    if (d_t == 128 && d_s == 128) return launch_bwd<128, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s);
+    if (d_t == 128 && d_s == 64) return launch_bwd<128, 64, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s);
+    return launch_bwd<64, 128, TEACHER>(q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s);
 }
 
-// Shared body of the three backward entry points.  `parts` selects the
-// kernels; the gradient pointers a part does not write may be NULL.
+// Bytes of workspace beyond the status word that the key-owner kernel needs
+// for its per-query-head dK partials when key heads are grouped (required).
+size_t dk_group_bytes(long long BH, int N_K, int d_t, int d_s, int H, int H_kt, int H_ks, bool teacher) {
+    size_t n = 0;
+    if (H_ks < H) n += (size_t)BH * N_K * d_s;
+    if (teacher && H_kt < H) n += (size_t)BH * N_K * d_t;
+    return n * sizeof(float);
+}
+
+// Shared body of the backward entry points.  `parts` selects the kernels; the
+// gradient pointers a part does not write may be NULL.  K_t and K_s have
+// H_kt, H_ks heads (dividing H); kv_len (per batch, nullable) marks padding.
 streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
-                           int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
-                           const float *kl, const float *lse_t, const float *lse_s, const float *dkl, float dloss,
-                           const float *dloss_dev, float *dq_s, float *dk_s, float *dq_t, float *dk_t,
-                           void *workspace, size_t workspace_bytes, void *stream, int parts) {
+                           int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s,
+                           int causal, const int *kv_len, const float *kl, const float *lse_t, const float *lse_s,
+                           const float *dkl, float dloss, const float *dloss_dev, float *dq_s, float *dk_s,
+                           float *dq_t, float *dk_t, void *workspace, size_t workspace_bytes, void *stream,
+                           int parts) {
     streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
     if (st != STREAMKL_OK) return st;
+    if ((st = check_heads(H, H_kt, H_ks, kv_len)) != STREAMKL_OK) return st;
     if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
     const bool want_dk = parts & kPartDK, want_dq = parts & kPartDQ;
     if (!(dloss == dloss)) return STREAMKL_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     const int BH = B * H;
+    const long long BKt = (long long)B * H_kt, BKs = (long long)B * H_ks;
     // Outputs with no elements may be NULL (an empty tensor has no storage).
     const bool dk_out = want_dk && (long long)BH * N_K > 0, dq_out = want_dq && (long long)BH * N_Q > 0;
     // the teacher pair of each part must be both given or both absent
@@ -256,12 +302,14 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     const bool teacher = dk_out ? dk_t != nullptr : dq_t != nullptr;
     if (dk_out && (!dk_s || (teacher && !dk_t))) return STREAMKL_ERR_INVALID_ARG;
     if (dq_out && (!dq_s || (teacher && !dq_t))) return STREAMKL_ERR_INVALID_ARG;
+    const size_t dk_part = want_dk ? dk_group_bytes(BH, N_K, d_t, d_s, H, H_kt, H_ks, teacher) : 0;
+    if (dk_part > 0 && workspace_bytes < kWorkspaceBytes + dk_part) return STREAMKL_ERR_WORKSPACE;
     if ((long long)BH * N_K == 0) return STREAMKL_OK;       // no keys (so no rows either): nothing to write
     if ((long long)BH * N_Q == 0) {                         // keys but no queries: every dK is zero
         if (want_dk) {
-            if (cudaMemsetAsync(dk_s, 0, (size_t)BH * N_K * d_s * sizeof(float), s) != cudaSuccess)
+            if (cudaMemsetAsync(dk_s, 0, (size_t)BKs * N_K * d_s * sizeof(float), s) != cudaSuccess)
                 return STREAMKL_ERR_CUDA;
-            if (teacher && cudaMemsetAsync(dk_t, 0, (size_t)BH * N_K * d_t * sizeof(float), s) != cudaSuccess)
+            if (teacher && cudaMemsetAsync(dk_t, 0, (size_t)BKt * N_K * d_t * sizeof(float), s) != cudaSuccess)
                 return STREAMKL_ERR_CUDA;
         }
         return STREAMKL_OK;
@@ -275,6 +323,7 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     BwdParams p;
     memset(&p, 0, sizeof p);
     p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
+    p.H = H; p.Hkt = H_kt; p.Hks = H_ks; p.kv_len = kv_len;
     p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
     p.out_t = scale_t * 0.69314718055994530942f;
     p.out_s = scale_s;
@@ -288,11 +337,22 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
     p.inv_scale_t = 1.0f / scale_t;
     p.inv_scale_s = 1.0f / scale_s;
     p.dq_s = dq_s; p.dk_s = dk_s; p.dq_t = dq_t; p.dk_t = dk_t;
+    DkOut out{dk_s, dk_t};
+    if (dk_part > 0) {               // grouped key heads: per-query-head partials in the workspace
+        float *part = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWorkspaceBytes);
+        if (H_ks < H) {
+            p.dk_s = part;
+            part += (size_t)BH * N_K * d_s;
+        }
+        if (teacher && H_kt < H) p.dk_t = part;
+    }
     p.qt_raw = q_t; p.kt_raw = k_t; p.qs_raw = q_s; p.ks_raw = k_s;
     p.st.word = static_cast<uint32_t *>(workspace);
     p.st.budget_ns = kWaitBudgetNs;
     p.splits = 1;
     if (want_dq) {
+        // dQ partials of key splits reuse the bytes after the status word: the
+        // dK partials there are summed (same stream) before the dQ kernel runs
         const long long rows = (long long)BH * N_Q;
         const int S = key_splits(BH, N_Q, N_K, causal);
         if (S > 1 && workspace_bytes >= kWorkspaceBytes + dq_split_bytes(S, rows, d_s, teacher ? d_t : 0)) {
@@ -301,8 +361,63 @@ streamkl_status bwd_common(const void *q_t, const void *k_t, const void *q_s, co
             p.part_t = p.part_s + (size_t)S * rows * d_s;
         }
     }
-    return teacher ? dispatch_bwd<true>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s)
-                   : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, s);
+    return teacher ? dispatch_bwd<true>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s)
+                   : dispatch_bwd<false>(d_t, d_s, q_t, k_t, q_s, k_s, N_Q, N_K, p, parts, out, s);
+}
+
+// Shared body of the forward entry points.  K_t and K_s have H_kt, H_ks heads
+// (dividing H); kv_len (per batch, nullable) marks padding.
+streamkl_status fwd_common(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                           int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s,
+                           int causal, const int *kv_len, float *kl, float *lse_t, float *lse_s, float *loss_mean,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
+    if (st != STREAMKL_OK) return st;
+    if ((st = check_heads(H, H_kt, H_ks, kv_len)) != STREAMKL_OK) return st;
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
+    if ((st = fwd_check_pointers(q_t, k_t, q_s, k_s, B, H, N_Q, kl, lse_t, lse_s)) != STREAMKL_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int BH = B * H;
+    const long long rows = (long long)BH * N_Q;
+    if (rows == 0) {
+        if (loss_mean) streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
+        return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
+    }
+    if ((st = check_device()) != STREAMKL_OK) return st;
+
+    CUtensorMap mqt, mkt, mqs, mks;
+    // Q boxes of 128 rows (one query tile), K boxes of 64 rows (one key tile)
+    if (!make_map(&mqt, q_t, d_t, N_Q, BH, 128) || !make_map(&mkt, k_t, d_t, N_K, B * H_kt, 64) ||
+        !make_map(&mqs, q_s, d_s, N_Q, BH, 128) || !make_map(&mks, k_s, d_s, N_K, B * H_ks, 64))
+        return STREAMKL_ERR_CUDA;
+    FwdParams p;
+    p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
+    p.H = H; p.Hkt = H_kt; p.Hks = H_ks; p.kv_len = kv_len;
+    p.n_qt = (N_Q + 127) / 128;
+    p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
+    p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s;
+    p.st.word = static_cast<uint32_t *>(workspace);
+    p.st.budget_ns = kWaitBudgetNs;
+    p.splits = 1;
+    p.part = nullptr;
+    {
+        const int S = key_splits(BH, N_Q, N_K, causal);
+        if (S > 1 && workspace_bytes >= kWorkspaceBytes + fwd_split_bytes(S, rows)) {
+            p.splits = S;
+            p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWorkspaceBytes);
+        }
+    }
+    if (d_t == 64 && d_s == 64) st = launch_fwd<64, 64>(mqt, mkt, mqs, mks, p, s);
+    else if (d_t == 128 && d_s == 128) st = launch_fwd<128, 128>(mqt, mkt, mqs, mks, p, s);
+    else if (d_t == 128 && d_s == 64) st = launch_fwd<128, 64>(mqt, mkt, mqs, mks, p, s);
+    else st = launch_fwd<64, 128>(mqt, mkt, mqs, mks, p, s);
+    if (st != STREAMKL_OK) return st;
+    if (loss_mean) {
+        streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, rows, (double)rows, 1.0, loss_mean);
+        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
+    }
+    return STREAMKL_OK;
 }
 
 // Self-test of the failure path: one warp waits, with the library's bounded
@@ -345,6 +460,16 @@ streamkl_status streamkl_selftest_timeout(void *workspace, size_t workspace_byte
 
 int streamkl_version(void) { return 100; }
 
+size_t streamkl_workspace_size_ex(int B, int H, int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, int causal,
+                                  int teacher_grads) {
+    const size_t base = streamkl_workspace_size(B, H, N_Q, N_K, d_t, d_s, causal);
+    if (B <= 0 || H <= 0 || N_K <= 0 || H_kt < 1 || H_ks < 1 || H % H_kt || H % H_ks) return base;
+    if ((d_t != 64 && d_t != 128) || (d_s != 64 && d_s != 128)) return base;
+    const size_t dk = dk_group_bytes((long long)B * H, N_K, d_t, d_s, H, H_kt, H_ks, teacher_grads != 0);
+    const size_t need = kWorkspaceBytes + ((dk + 255) / 256) * 256;
+    return std::max(base, need);
+}
+
 size_t streamkl_workspace_size(int B, int H, int N_Q, int N_K, int d_t, int d_s, int causal) {
     if (B <= 0 || H <= 0 || N_Q <= 0 || N_K <= 0 || (d_t != 64 && d_t != 128) || (d_s != 64 && d_s != 128))
         return kWorkspaceBytes;
@@ -386,58 +511,24 @@ streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int
     }
     if (code_out) *code_out = word;
     if (cudaPeekAtLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
-    return (word & kStatusTimeout) ? STREAMKL_ERR_TIMEOUT : STREAMKL_OK;
+    if (word & kStatusTimeout) return STREAMKL_ERR_TIMEOUT;
+    return (word & kStatusBadLength) ? STREAMKL_ERR_INVALID_ARG : STREAMKL_OK;
 }
 
 streamkl_status streamkl_fwd(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
                              int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s, int causal,
                              float *kl, float *lse_t, float *lse_s, float *loss_mean, void *workspace,
                              size_t workspace_bytes, void *stream) {
-    streamkl_status st = check_shape(B, H, N_Q, N_K, d_t, d_s, causal, scale_t, scale_s);
-    if (st != STREAMKL_OK) return st;
-    if (!workspace || workspace_bytes < kWorkspaceBytes) return STREAMKL_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return STREAMKL_ERR_INVALID_ARG;
-    if ((st = fwd_check_pointers(q_t, k_t, q_s, k_s, B, H, N_Q, kl, lse_t, lse_s)) != STREAMKL_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    const int BH = B * H;
-    const long long rows = (long long)BH * N_Q;
-    if (rows == 0) {
-        if (loss_mean) streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, 0, 1.0, 1.0, loss_mean);
-        return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_CUDA;
-    }
-    if ((st = check_device()) != STREAMKL_OK) return st;
+    return fwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, nullptr, kl,
+                      lse_t, lse_s, loss_mean, workspace, workspace_bytes, stream);
+}
 
-    CUtensorMap mqt, mkt, mqs, mks;
-    // Q boxes of 128 rows (one query tile), K boxes of 64 rows (one key tile)
-    if (!make_map(&mqt, q_t, d_t, N_Q, BH, 128) || !make_map(&mkt, k_t, d_t, N_K, BH, 64) ||
-        !make_map(&mqs, q_s, d_s, N_Q, BH, 128) || !make_map(&mks, k_s, d_s, N_K, BH, 64))
-        return STREAMKL_ERR_CUDA;
-    FwdParams p;
-    p.BH = BH; p.N_Q = N_Q; p.N_K = N_K; p.causal = causal;
-    p.n_qt = (N_Q + 127) / 128;
-    p.ct = scale_t * kLog2e; p.cs = scale_s * kLog2e;
-    p.kl = kl; p.lse_t = lse_t; p.lse_s = lse_s;
-    p.st.word = static_cast<uint32_t *>(workspace);
-    p.st.budget_ns = kWaitBudgetNs;
-    p.splits = 1;
-    p.part = nullptr;
-    {
-        const int S = key_splits(BH, N_Q, N_K, causal);
-        if (S > 1 && workspace_bytes >= kWorkspaceBytes + fwd_split_bytes(S, rows)) {
-            p.splits = S;
-            p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWorkspaceBytes);
-        }
-    }
-    if (d_t == 64 && d_s == 64) st = launch_fwd<64, 64>(mqt, mkt, mqs, mks, p, s);
-    else if (d_t == 128 && d_s == 128) st = launch_fwd<128, 128>(mqt, mkt, mqs, mks, p, s);
-    else if (d_t == 128 && d_s == 64) st = launch_fwd<128, 64>(mqt, mkt, mqs, mks, p, s);
-    else st = launch_fwd<64, 128>(mqt, mkt, mqs, mks, p, s);
-    if (st != STREAMKL_OK) return st;
-    if (loss_mean) {
-        streamkl_mean_kernel<<<kMeanCtas, kMeanThreads, 0, s>>>(kl, rows, (double)rows, 1.0, loss_mean);
-        if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
-    }
-    return STREAMKL_OK;
+streamkl_status streamkl_fwd_ex(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                                int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s,
+                                int causal, const int *kv_len, float *kl, float *lse_t, float *lse_s,
+                                float *loss_mean, void *workspace, size_t workspace_bytes, void *stream) {
+    return fwd_common(q_t, k_t, q_s, k_s, B, H, H_kt, H_ks, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kv_len, kl,
+                      lse_t, lse_s, loss_mean, workspace, workspace_bytes, stream);
 }
 
 
@@ -447,7 +538,8 @@ streamkl_status streamkl_bwd(const void *q_t, const void *k_t, const void *q_s, 
                              const float *kl, const float *lse_t, const float *lse_s, const float *dkl, float dloss,
                              float *dq_s, float *dk_s, float *dq_t, float *dk_t, void *workspace,
                              size_t workspace_bytes, void *stream) {
-    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, nullptr, kl, lse_t,
+                      lse_s, dkl,
                       dloss, nullptr, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes, stream, kPartDK | kPartDQ);
 }
 
@@ -456,7 +548,8 @@ streamkl_status streamkl_bwd_dk(const void *q_t, const void *k_t, const void *q_
                                 const float *kl, const float *lse_t, const float *lse_s, const float *dkl,
                                 float dloss, float *dk_s, float *dk_t, void *workspace, size_t workspace_bytes,
                                 void *stream) {
-    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, nullptr, kl, lse_t,
+                      lse_s, dkl,
                       dloss, nullptr, nullptr, dk_s, nullptr, dk_t, workspace, workspace_bytes, stream, kPartDK);
 }
 
@@ -465,7 +558,8 @@ streamkl_status streamkl_bwd_dq(const void *q_t, const void *k_t, const void *q_
                                 const float *kl, const float *lse_t, const float *lse_s, const float *dkl,
                                 float dloss, float *dq_s, float *dq_t, void *workspace, size_t workspace_bytes,
                                 void *stream) {
-    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, nullptr, kl, lse_t,
+                      lse_s, dkl,
                       dloss, nullptr, dq_s, nullptr, dq_t, nullptr, workspace, workspace_bytes, stream, kPartDQ);
 }
 
@@ -476,9 +570,25 @@ streamkl_status streamkl_bwd_dloss_device(const void *q_t, const void *k_t, cons
                                           float *dk_s, float *dq_t, float *dk_t, void *workspace,
                                           size_t workspace_bytes, void *stream) {
     if (!dkl && !dloss_dev) return STREAMKL_ERR_INVALID_ARG;
-    return bwd_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kl, lse_t, lse_s, dkl,
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, nullptr, kl, lse_t,
+                      lse_s, dkl,
                       dloss_scale, dkl ? nullptr : dloss_dev, dq_s, dk_s, dq_t, dk_t, workspace, workspace_bytes,
                       stream, kPartDK | kPartDQ);
+}
+
+streamkl_status streamkl_bwd_ex(const void *q_t, const void *k_t, const void *q_s, const void *k_s, int B, int H,
+                                int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, float scale_t, float scale_s,
+                                int causal, const int *kv_len, const float *kl, const float *lse_t,
+                                const float *lse_s, const float *dkl, float dloss, const float *dloss_dev,
+                                float *dq_s, float *dk_s, float *dq_t, float *dk_t, int parts, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (parts < 1 || parts > (kPartDK | kPartDQ)) return STREAMKL_ERR_INVALID_ARG;
+    // the part not asked for writes nothing: its pointers are ignored
+    if (!(parts & kPartDK)) dk_s = dk_t = nullptr;
+    if (!(parts & kPartDQ)) dq_s = dq_t = nullptr;
+    return bwd_common(q_t, k_t, q_s, k_s, B, H, H_kt, H_ks, N_Q, N_K, d_t, d_s, scale_t, scale_s, causal, kv_len, kl,
+                      lse_t, lse_s, dkl, dloss, dkl ? nullptr : dloss_dev, dq_s, dk_s, dq_t, dk_t, workspace,
+                      workspace_bytes, stream, parts);
 }
 
 streamkl_status streamkl_loss_mean(const float *kl, long long n_rows, float *loss_mean, void *stream) {

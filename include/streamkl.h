@@ -171,10 +171,74 @@ streamkl_status streamkl_loss_reduce(const float *kl, long long n_rows, double f
 streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream` and returns STREAMKL_ERR_TIMEOUT if a kernel of an
- * earlier call on this workspace gave up on a bounded wait, STREAMKL_ERR_CUDA
- * if the stream reports a CUDA error, else STREAMKL_OK.  `code_out` (host
- * pointer, nullable) receives the raw device status word (0 = clean). */
+ * earlier call on this workspace gave up on a bounded wait,
+ * STREAMKL_ERR_INVALID_ARG if a kernel met a per-batch key length outside
+ * [0, N_K] (streamkl_fwd_ex / streamkl_bwd_ex; the length was clamped),
+ * STREAMKL_ERR_CUDA if the stream reports a CUDA error, else STREAMKL_OK.
+ * `code_out` (host pointer, nullable) receives the raw device status word
+ * (0 = clean; bit 0 timeout, bit 1 bad length, bits 8..15 which wait). */
 streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int *code_out);
+
+/*
+ * Padded batches and grouped key heads.
+ * Source: the abstract of "StreamKL: ..." names sparse-attention LLM training
+ * and long-context distillation as the uses; both feed batches of sequences
+ * padded to a common length and models whose keys have fewer heads than their
+ * queries.  The pages give no formula for either, so these take the plain
+ * readings:
+ *  - K_t is [B, H_kt, N_K, d_t] and K_s is [B, H_ks, N_K, d_s], H_kt and H_ks
+ *    each >= 1 and dividing H (else STREAMKL_ERR_INVALID_ARG); query head h of
+ *    batch b reads key head b * H_k + h / (H / H_k).  Q_t, Q_s and every
+ *    per-row vector keep H heads.  dk_t and dk_s have their key tensor's shape:
+ *    a key head's gradient is the sum over the query heads that read it
+ *    (computed as one partial per query head in the workspace, then summed in
+ *    a fixed order, so the result is the same run to run).
+ *  - kv_len: DEVICE int32 [B] (4-byte aligned), or NULL for no padding.  Key j
+ *    is visible to row i of batch b iff the causal rule above allows it AND
+ *    j < kv_len[b] (the causal diagonal stays at N_K - N_Q).  A row with no
+ *    visible key (kv_len[b] = 0) gets kl = 0, lse_t = lse_s = -inf and zero
+ *    gradients; keys at and past kv_len[b] get zero dK rows.  Lengths are read
+ *    on the device: one outside [0, N_K] is clamped to it and sets a bit that
+ *    streamkl_check() reports as STREAMKL_ERR_INVALID_ARG.
+ * With H_kt = H_ks = H and kv_len = NULL these are streamkl_fwd, streamkl_bwd.
+ */
+
+/* Workspace bytes for streamkl_fwd_ex / streamkl_bwd_ex on the current
+ * device: streamkl_workspace_size plus, for the key gradients of grouped key
+ * heads, B * H * N_K floats per grouped side (d_s for the student; d_t for
+ * the teacher when teacher_grads != 0).  That part is REQUIRED by
+ * streamkl_bwd_ex (a smaller workspace is STREAMKL_ERR_WORKSPACE); the rest
+ * only enables key splits, as for streamkl_bwd. */
+size_t streamkl_workspace_size_ex(int B, int H, int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s, int causal,
+                                  int teacher_grads);
+
+/* streamkl_fwd with grouped key heads and padding (see above).  Arguments,
+ * results and errors otherwise as streamkl_fwd; loss_mean is the mean over all
+ * B*H*N_Q rows (rows of padded queries included: leave them out of a mean
+ * with the per-row kl and weights). */
+streamkl_status streamkl_fwd_ex(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                int B, int H, int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s,
+                                float scale_t, float scale_s, int causal, const int *kv_len,
+                                float *kl, float *lse_t, float *lse_s, float *loss_mean,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* streamkl_bwd with grouped key heads and padding (see above), taking every
+ * form of the upstream gradient and either half of the backward:
+ *   g_i = dkl[i]                      if dkl != NULL
+ *   g_i = dloss * (*dloss_dev)        else if dloss_dev != NULL (device scalar)
+ *   g_i = dloss / (B*H*N_Q)           otherwise
+ * parts: 1 = key gradients (dk_s, dk_t), 2 = query gradients (dq_s, dq_t),
+ * 3 = both (other values: STREAMKL_ERR_INVALID_ARG); the pointers of a part
+ * not asked for are ignored.  The teacher pair of a part asked for must be
+ * both NULL or both given (for parts = 3: all four teacher pointers alike).
+ * kl, lse_t, lse_s must come from streamkl_fwd_ex with the same arguments. */
+streamkl_status streamkl_bwd_ex(const void *q_t, const void *k_t, const void *q_s, const void *k_s,
+                                int B, int H, int H_kt, int H_ks, int N_Q, int N_K, int d_t, int d_s,
+                                float scale_t, float scale_s, int causal, const int *kv_len,
+                                const float *kl, const float *lse_t, const float *lse_s,
+                                const float *dkl, float dloss, const float *dloss_dev,
+                                float *dq_s, float *dk_s, float *dq_t, float *dk_t, int parts,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Forward with no device memory from the caller beyond inputs and outputs.
