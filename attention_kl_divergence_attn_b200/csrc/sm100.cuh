@@ -363,12 +363,11 @@ __device__ __forceinline__ float lg2(float x) {
     return y;
 }
 
-// One 4-byte shared-memory load that the compiler may not merge with its
-// neighbours: when every thread of a warp reads the same address it costs a
-// single wavefront, where a merged 16-byte broadcast load costs several.
-__device__ __forceinline__ float ld_shared_f32(const float *p) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
+// One 16-byte shared-memory load issued exactly here (`p` 16-byte aligned).
+__device__ __forceinline__ float4 ld_shared_v4(const float *p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p)));
     return v;
 }
 

@@ -217,12 +217,17 @@ streamkl_status launch_bwd(const void *q_t, const void *k_t, const void *q_s, co
         // the items, overlapping each item's start with the previous one's end)
         // is faster; at the register limit (teacher and student K in shared
         // memory) one CTA per item keeps the inner loop faster.
-        auto kdkv = CK::K_TMEM ? streamkl_bwd_dkv_persistent_kernel<DT, DS, TEACHER>
-                    : (p.kv_len ? streamkl_bwd_dkv_kernel<DT, DS, TEACHER, true>
-                                : streamkl_bwd_dkv_kernel<DT, DS, TEACHER, false>);
-        if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
-        const long long grid = CK::K_TMEM ? std::min<long long>(items, std::max(1, sm_count())) : items;
-        kdkv<<<(unsigned)grid, CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        if constexpr (CK::K_TMEM) {
+            auto kdkv = streamkl_bwd_dkv_persistent_kernel<DT, DS, TEACHER>;
+            if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+            const long long grid = std::min<long long>(items, std::max(1, sm_count()));
+            kdkv<<<(unsigned)grid, CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        } else {
+            auto kdkv = p.kv_len ? streamkl_bwd_dkv_kernel<DT, DS, TEACHER, true>
+                                 : streamkl_bwd_dkv_kernel<DT, DS, TEACHER, false>;
+            if (set_smem(kdkv, CK::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+            kdkv<<<(unsigned)items, CK::THREADS, CK::SMEM, stream>>>(mqt, mkt, mqs, mks, p);
+        }
         if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
         // grouped key heads: each key head's gradient is its group's partials summed in order
         streamkl_status st = STREAMKL_OK;
