@@ -30,7 +30,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libstreamkl.so")
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "device wait timeout",
-          5: "workspace"}
+          5: "workspace", 6: "access outside a tensor (bounds-checked build)"}
 
 
 class StreamKLError(RuntimeError):

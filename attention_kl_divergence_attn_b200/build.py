@@ -1,5 +1,10 @@
 """Builds libstreamkl.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
+Also builds libstreamkl_checked.so, the same library with every TMA coordinate
+and global index checked against its tensor (STREAMKL_CHECK_BOUNDS): a debug
+build for tests, which report an access outside a tensor through the status
+word instead of faulting.
+
 Usage: python -m attention_kl_divergence_attn_b200.build [--force]
 """
 from __future__ import annotations
@@ -15,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libstreamkl.so")
+CHECKED_LIB = os.path.join(PKG, "libstreamkl_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -36,26 +42,29 @@ def sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, os.path.join(CSRC, "streamkl.cu"), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Builds libstreamkl.so, or with `checked` the bounds-checked debug build."""
+    lib = CHECKED_LIB if checked else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".{os.getpid()}.tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DSTREAMKL_CHECK_BOUNDS"] if checked else []), "-I", INCLUDE,
+           os.path.join(CSRC, "streamkl.cu"), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, checked=True))

@@ -285,12 +285,13 @@ constexpr int kBwdChunk = 64 / kBwdHalves;
 // stores the tile with 16-byte loads and stores, 32 / (NCOLS / 4) whole row
 // segments per instruction, so every global store covers complete 64- or
 // 128-byte runs.  `dst` points at column 0 of row row0 and is 16-byte
-// aligned, as is `ld` * 4 bytes, the row stride.
+// aligned, as is `ld` * 4 bytes, the row stride.  `lim` is one past the end
+// of the output tensor (checked in the bounds-checked build).
 constexpr int kDrainPad = 4;
 
 template <int NCOLS>
 __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *dst, size_t ld, int nvalid,
-                                           float *stage, int lane, bool zero) {
+                                           float *stage, int lane, bool zero, const float *lim, uint32_t *word) {
     static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
     constexpr int SP = NCOLS + kDrainPad, V = NCOLS / 4, RPI = 32 / V;
     float4 *mine = reinterpret_cast<float4 *>(stage + lane * SP);
@@ -310,7 +311,7 @@ __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *d
 #pragma unroll
     for (int j = 0; j < 32 / RPI; ++j) {
         const int r = j * RPI + rr;
-        if (r < nvalid)
+        if (r < nvalid && bound_ok(dst + (size_t)r * ld + c4 + 4 <= lim, word, kSiteDrain))
             *reinterpret_cast<float4 *>(dst + (size_t)r * ld + c4) =
                 *reinterpret_cast<const float4 *>(stage + r * SP + c4);
     }
@@ -322,7 +323,8 @@ __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *d
 // `valid`), straight from registers: 32-byte stores when `dst` is 32-byte aligned (whole sectors),
 // else 16-byte stores.
 template <int NCOLS>
-__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool valid, bool zero) {
+__device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *dst, bool valid, bool zero,
+                                          const float *lim, uint32_t *word) {
     static_assert(NCOLS == 16 || NCOLS == 32, "16 or 32 columns");
     const bool a32 = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
 #pragma unroll
@@ -332,7 +334,7 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, float scale, float *ds
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[k] = zero ? 0.f : v[k] * scale;
-        if (valid) {
+        if (valid && bound_ok(dst + c + 16 <= lim, word, kSiteDrain)) {
             if (a32) {
                 st_global_v8(dst + c, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
                 st_global_v8(dst + c + 8, v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
@@ -419,6 +421,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tensors behind the four maps (bounds-checked build)
+    const MapDims mdQt{DT, p.N_Q, p.BH}, mdQs{DS, p.N_Q, p.BH};
+    const MapDims mdKt{DT, p.N_K, p.BH / p.H * p.Hkt}, mdKs{DS, p.N_K, p.BH / p.H * p.Hks};
     const int kt_idx = (int)(blockIdx.x / p.BH);   // low key tiles see the most queries: run them first
     const int bh = (int)(blockIdx.x % p.BH);
     const int k0 = kt_idx * C::BN;
@@ -434,6 +439,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const int nk = key_count(p.kv_len, bh / p.H, p.N_K, p.st.word, threadIdx.x == 0 && kt_idx == 0);
         if (k0 >= nk) {
             const int rows = min(C::BN, p.N_K - k0);
+            if (!bound_ok(bh < p.BH && k0 >= 0 && rows > 0, p.st.word, kSiteZero)) return;
             float4 *ds4 = reinterpret_cast<float4 *>(p.dk_s + ((size_t)bh * p.N_K + k0) * DS);
             for (int e = threadIdx.x; e < rows * DS / 4; e += C::THREADS) ds4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (TEACHER) {
@@ -467,19 +473,19 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 prefetch_tmap(&mKt); prefetch_tmap(&mKs);
                 mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
+                for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt, mdKt, p.st.word);
 #pragma unroll
-                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
+                for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks, mdKs, p.st.word);
             }
             prefetch_tmap(&mQt); prefetch_tmap(&mQs);
             if (n_qt > 0) {
                 mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh, mdQt, p.st.word);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh, mdQs, p.st.word);
             }
         }
     } else if (warp == 1) {
@@ -512,8 +518,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     if constexpr (C::K_TMEM) {
         if (warp >= 2) {
             const int wg = (warp - 2) >> 2, sub = warp & 3;
-            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bkt, p.N_K, k0, wg, sub, lane);
-            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bks, p.N_K, k0, wg, sub, lane);
+            resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, bkt, p.N_K, k0, wg, sub, lane, mdKt.n2, p.st.word);
+            resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, bks, p.N_K, k0, wg, sub, lane, mdKs.n2, p.st.word);
             tmem_st_wait();
         }
         tc_fence_before();
@@ -534,7 +540,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             for (int h = 0; h < 2; ++h) {
                 const int i = q0 + lane + 32 * h;
                 v[h] = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
-                if (t < n_qt && i < p.N_Q) {
+                if (t < n_qt && i < p.N_Q && bound_ok(bh < p.BH && i >= 0, p.st.word, kSiteConst)) {
                     const size_t r = (size_t)bh * p.N_Q + i;
                     v[h].x = ld_now(p.lse_t + r);
                     v[h].y = ld_now(p.lse_s + r);
@@ -559,10 +565,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::QBLK, &mQt, &bar_qfull[s], b * 64, q0, bh);
+                    tma_load_3d(st + b * C::QBLK, &mQt, &bar_qfull[s], b * 64, q0, bh, mdQt, p.st.word);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh);
+                    tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh, mdQs, p.st.word);
             }
             float *ktab = reinterpret_cast<float *>(st + C::GK), *gtab = ktab + C::BM;
 #pragma unroll
@@ -713,15 +719,18 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             // a padding key: its row is zero (the length is read again here rather
             // than kept live through the tile loop)
             const bool pad = PAD && gk >= key_count(p.kv_len, bh / p.H, p.N_K, nullptr, false);
+            const size_t nk_all = (size_t)p.BH * p.N_K;   // rows of the output (or its per-head partial)
             drain_rows<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + r0 * DS + wg * HS, DS, nvalid,
-                           stage, lane, pad);
+                           stage, lane, pad, p.dk_s + nk_all * DS, p.st.word);
             if (TEACHER)
                 drain_rows<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + r0 * DT + wg * HT, DT,
-                               nvalid, stage, lane, pad);
+                               nvalid, stage, lane, pad, p.dk_t + nk_all * DT, p.st.word);
         } else if (n_qt == 0 && gk < p.N_K && wg == 0) {
             const size_t r = (size_t)bh * p.N_K + gk;
-            for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
-            if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[r * DT + c] = 0.f;
+            if (bound_ok(r < (size_t)p.BH * p.N_K, p.st.word, kSiteZero)) {
+                for (int c = 0; c < DS; ++c) p.dk_s[r * DS + c] = 0.f;
+                if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[r * DT + c] = 0.f;
+            }
         }
     }
 
@@ -777,6 +786,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tensors behind the four maps (bounds-checked build)
+    const MapDims mdQt{DT, p.N_Q, p.BH}, mdQs{DS, p.N_Q, p.BH};
+    const MapDims mdKt{DT, p.N_K, p.BH / p.H * p.Hkt}, mdKs{DS, p.N_K, p.BH / p.H * p.Hks};
     const int off = p.N_K - p.N_Q;
     const int n_qt_all = (p.N_Q + C::BM - 1) / C::BM;
     const int n_items = p.BH * p.n_tiles;
@@ -821,24 +833,24 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 if (!C::K_TMEM) {
                     mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt, mdKt, p.st.word);
 #pragma unroll
-                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks, mdKs, p.st.word);
                 } else if (C::K_STAGED) {
                     mbar_expect_tx(&bar_kst, C::KST_BYTES);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, k0, bkt);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, k0, bkt, mdKt, p.st.word);
 #pragma unroll
                     for (int b = 0; b < DS / 64; ++b)
-                        tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, k0, bks);
+                        tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, k0, bks, mdKs, p.st.word);
                 }
                 mbar_expect_tx(&bar_qfull[0], C::STAGE_TMA);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+                    tma_load_3d(sQ + b * C::QBLK, &mQt, &bar_qfull[0], b * 64, first_qt * C::BM, bh, mdQt, p.st.word);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
-                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh);
+                    tma_load_3d(sQ + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[0], b * 64, first_qt * C::BM, bh, mdQs, p.st.word);
             }
         }
     } else if (warp == 1) {
@@ -904,10 +916,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             const int kbt = key_head(kst_bh, p.H, p.Hkt), kbs = key_head(kst_bh, p.H, p.Hks);
 #pragma unroll
             for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kbt);
+                tma_load_3d(sKst + b * C::KBLK, &mKt, &bar_kst, b * 64, kst_k0, kbt, mdKt, p.st.word);
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kbs);
+                tma_load_3d(sKst + C::BN * DT * 2 + b * C::KBLK, &mKs, &bar_kst, b * 64, kst_k0, kbs, mdKs, p.st.word);
             ++kst_n;
             ++kst_r;
             kst_find();
@@ -936,9 +948,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     mbar_expect_tx(&bar_k, C::KT_BYTES + C::KS_BYTES);
                     const int bkt = key_head(bh, p.H, p.Hkt), bks = key_head(bh, p.H, p.Hks);
 #pragma unroll
-                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt);
+                    for (int b = 0; b < DT / 64; ++b) tma_load_3d(sKt + b * C::KBLK, &mKt, &bar_k, b * 64, k0, bkt, mdKt, p.st.word);
 #pragma unroll
-                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks);
+                    for (int b = 0; b < DS / 64; ++b) tma_load_3d(sKs + b * C::KBLK, &mKs, &bar_k, b * 64, k0, bks, mdKs, p.st.word);
                 }
             }
             if (!C::K_TMEM) ++k_issued;
@@ -966,7 +978,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 for (int h = 0; h < 2; ++h) {
                     const int i = q0 + lane + 32 * h;
                     v[h] = make_float4(0.f, 0.f, 0.f, 0.f);        // rows past N_Q: g = 0, so dS = 0
-                    if (t < n_qt && i < p.N_Q) {
+                    if (t < n_qt && i < p.N_Q && bound_ok(bh < p.BH && i >= 0, p.st.word, kSiteConst)) {
                         const size_t rr = (size_t)bh * p.N_Q + i;
                         v[h].x = ld_now(p.lse_t + rr);
                         v[h].y = ld_now(p.lse_s + rr);
@@ -991,10 +1003,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     mbar_expect_tx(&bar_qfull[s], C::STAGE_TMA);
 #pragma unroll
                     for (int b = 0; b < DT / 64; ++b)
-                        tma_load_3d(st + b * C::QBLK, &mQt, &bar_qfull[s], b * 64, q0, bh);
+                        tma_load_3d(st + b * C::QBLK, &mQt, &bar_qfull[s], b * 64, q0, bh, mdQt, p.st.word);
 #pragma unroll
                     for (int b = 0; b < DS / 64; ++b)
-                        tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh);
+                        tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh, mdQs, p.st.word);
                 }
                 float *ktab = reinterpret_cast<float *>(st + C::GK), *gtab = ktab + C::BM;
 #pragma unroll
@@ -1148,8 +1160,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 tile_rows_to_tmem<DS>(lane_base + C::TMEM_KS, sKst + C::BN * DT * 2, wg, row);
             } else {
                 tc_fence_after();
-                resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, key_head(bh, p.H, p.Hkt), p.N_K, k0, wg, sub, lane);
-                resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, key_head(bh, p.H, p.Hks), p.N_K, k0, wg, sub, lane);
+                resident_to_tmem<DT>(tmem, C::TMEM_KT, p.kt_raw, key_head(bh, p.H, p.Hkt), p.N_K, k0, wg, sub, lane, mdKt.n2, p.st.word);
+                resident_to_tmem<DS>(tmem, C::TMEM_KS, p.ks_raw, key_head(bh, p.H, p.Hks), p.N_K, k0, wg, sub, lane, mdKs.n2, p.st.word);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -1171,8 +1183,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             if (n_qt == 0) {
                 if (gk < p.N_K && wg == 0) {       // no visible query: dK = 0
                     const size_t rr = (size_t)bh * p.N_K + gk;
-                    for (int c = 0; c < DS; ++c) p.dk_s[rr * DS + c] = 0.f;
-                    if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[rr * DT + c] = 0.f;
+                    if (bound_ok(rr < (size_t)p.BH * p.N_K, p.st.word, kSiteZero)) {
+                        for (int c = 0; c < DS; ++c) p.dk_s[rr * DS + c] = 0.f;
+                        if (TEACHER) for (int c = 0; c < DT; ++c) p.dk_t[rr * DT + c] = 0.f;
+                    }
                 }
             } else {
                 if (C::K_TMEM && !k_ready && !k_to_tmem(it, k0, bh)) { ok = false; break; }
@@ -1229,11 +1243,12 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 const bool pad = gk >= key_count(p.kv_len, bh / p.H, p.N_K, nullptr, false);   // zero row
                 const size_t grow = (size_t)bh * p.N_K + gk;
                 constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
+                const size_t nk_all = (size_t)p.BH * p.N_K;   // rows of the output (or its per-head partial)
                 drain_row<HS>(lane_base + C::TMEM_DKS + wg * HS, p.out_s * gs, p.dk_s + grow * DS + wg * HS, valid,
-                              pad);
+                              pad, p.dk_s + nk_all * DS, p.st.word);
                 if (TEACHER)
                     drain_row<HT>(lane_base + C::TMEM_DKT + wg * HT, p.out_t * gs, p.dk_t + grow * DT + wg * HT, valid,
-                                  pad);
+                                  pad, p.dk_t + nk_all * DT, p.st.word);
                 tc_fence_before();
                 g0 += n_qt;
                 ++it;
@@ -1298,6 +1313,9 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tensors behind the four maps (bounds-checked build)
+    const MapDims mdQt{DT, p.N_Q, p.BH}, mdQs{DS, p.N_Q, p.BH};
+    const MapDims mdKt{DT, p.N_K, p.BH / p.H * p.Hkt}, mdKs{DS, p.N_K, p.BH / p.H * p.Hks};
     // heaviest causal query tiles first; the key splits of a tile are adjacent
     const int lin = (int)(blockIdx.x / p.BH);
     const int split = lin % p.splits;
@@ -1339,18 +1357,18 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             prefetch_tmap(&mQt); prefetch_tmap(&mQs);
             mbar_expect_tx(&bar_q, C::QT_BYTES + C::QS_BYTES);
 #pragma unroll
-            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh);
+            for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::QBLK, &mQt, &bar_q, b * 64, q0, bh, mdQt, p.st.word);
 #pragma unroll
-            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh);
+            for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::QBLK, &mQs, &bar_q, b * 64, q0, bh, mdQs, p.st.word);
         }
         if (n_kt > 0) {
             mbar_expect_tx(&bar_kfull[0], C::STAGE_BYTES);
 #pragma unroll
             for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, kt_lo * C::BN, bkt);
+                tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, kt_lo * C::BN, bkt, mdKt, p.st.word);
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, kt_lo * C::BN, bks);
+                tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, kt_lo * C::BN, bks, mdKs, p.st.word);
         }
     }
     if (warp == 1) {
@@ -1365,8 +1383,8 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     if constexpr (C::Q_TMEM) {
         if (warp >= 2) {
             const int wg = (warp - 2) >> 2, sub = warp & 3;
-            resident_to_tmem<DT>(tmem, C::TMEM_QT, p.qt_raw, bh, p.N_Q, q0, wg, sub, lane);
-            resident_to_tmem<DS>(tmem, C::TMEM_QS, p.qs_raw, bh, p.N_Q, q0, wg, sub, lane);
+            resident_to_tmem<DT>(tmem, C::TMEM_QT, p.qt_raw, bh, p.N_Q, q0, wg, sub, lane, mdQt.n2, p.st.word);
+            resident_to_tmem<DS>(tmem, C::TMEM_QS, p.qs_raw, bh, p.N_Q, q0, wg, sub, lane, mdQs.n2, p.st.word);
             tmem_st_wait();
         }
         tc_fence_before();
@@ -1386,11 +1404,11 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt, mdKt, p.st.word);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
-                                bks);
+                                bks, mdKs, p.st.word);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -1522,11 +1540,14 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             }
             constexpr int HS = DS / C::NWG, HT = DT / C::NWG;
             // the row's g was left out of dS; no key tile: nothing was accumulated
+            const size_t nq_all = (size_t)p.splits * p.BH * p.N_Q;   // rows of the output, or of all partials
             drain_rows<HS>(lane_base + C::TMEM_DQS + wg * HS, p.out_s * g, dst_s + r0 * DS + wg * HS, DS, nvalid,
-                           stage, lane, n_kt == 0);
+                           stage, lane, n_kt == 0, dst_s + (p.splits > 1 ? nq_all : (size_t)p.BH * p.N_Q) * DS,
+                           p.st.word);
             if (TEACHER)
                 drain_rows<HT>(lane_base + C::TMEM_DQT + wg * HT, p.out_t * g, dst_t + r0 * DT + wg * HT, DT, nvalid,
-                               stage, lane, n_kt == 0);
+                               stage, lane, n_kt == 0,
+                               dst_t + (p.splits > 1 ? nq_all : (size_t)p.BH * p.N_Q) * DT, p.st.word);
         }
     }
 

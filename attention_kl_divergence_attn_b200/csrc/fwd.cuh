@@ -274,6 +274,9 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tensors behind the four maps (bounds-checked build)
+    const MapDims mdQt{DT, p.N_Q, p.BH}, mdQs{DS, p.N_Q, p.BH};
+    const MapDims mdKt{DT, p.N_K, p.BH / p.H * p.Hkt}, mdKs{DS, p.N_K, p.BH / p.H * p.Hks};
     // heaviest (latest) causal query tiles first; with key splits, the splits
     // of one query tile are adjacent in launch order
     const int lin = (int)(blockIdx.x / p.BH);
@@ -311,18 +314,18 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
         prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
         mbar_expect_tx(&bar_q, C::Q_BYTES);
 #pragma unroll
-        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh);
+        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, q0, bh, mdQt, p.st.word);
 #pragma unroll
-        for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh);
+        for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, q0, bh, mdQs, p.st.word);
         for (int kt = 0; kt < min(1, n_kt); ++kt) {
             uint8_t *st = sK + kt * C::STAGE_BYTES;
             mbar_expect_tx(&bar_kfull[kt], C::STAGE_BYTES);
 #pragma unroll
             for (int b = 0; b < DT / 64; ++b)
-                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bkt);
+                tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bkt, mdKt, p.st.word);
 #pragma unroll
             for (int b = 0; b < DS / 64; ++b)
-                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bks);
+                tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[kt], b * 64, (kt_lo + kt) * C::BN, bks, mdKs, p.st.word);
         }
     }
     if (warp == 1) {
@@ -347,11 +350,11 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < DT / 64; ++b)
-                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt);
+                    tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN, bkt, mdKt, p.st.word);
 #pragma unroll
                 for (int b = 0; b < DS / 64; ++b)
                     tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64, (kt_lo + kt) * C::BN,
-                                bks);
+                                bks, mdKs, p.st.word);
                 issued = kt + 1;
             }
             if (*abort_v) {
@@ -456,7 +459,8 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                                             merge[o][4][row]});
             }
         }
-        if (wg == 0 && grow < p.N_Q && !*abort_v) {
+        if (wg == 0 && grow < p.N_Q && !*abort_v &&
+            bound_ok(bh < p.BH && split < p.splits, p.st.word, kSiteRowOut)) {
             const size_t r = (size_t)bh * p.N_Q + grow;
             if (p.splits > 1) {
                 const size_t rows = (size_t)p.BH * p.N_Q, fs = (size_t)p.splits * rows;

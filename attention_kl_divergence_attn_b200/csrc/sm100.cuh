@@ -17,7 +17,44 @@ namespace skl {
 enum : uint32_t {
     kStatusTimeout = 1u << 0,   // some bounded wait gave up
     kStatusBadLength = 1u << 1, // a per-batch key length outside [0, N_K] (clamped)
+    kStatusBounds = 1u << 2,    // bounds-checked build: an access outside its tensor (skipped)
     kStatusWhoShift = 8,        // bits 8..15: which wait (role-specific id)
+    kStatusSiteShift = 16,      // bits 16..23: which checked access (bounds-checked build)
+};
+
+// ---------------------------------------------------------------- bounds-checked build
+// Built with STREAMKL_CHECK_BOUNDS (libstreamkl_checked.so), every TMA
+// coordinate and every global index that the kernels compute is checked
+// against its tensor before the access; a violation skips the access and ORs
+// kStatusBounds and the site's id into the status word (nothing traps, and a
+// skipped copy ends in a bounded wait that gives up).  Otherwise the checks
+// compile to nothing.
+#ifdef STREAMKL_CHECK_BOUNDS
+constexpr bool kCheckBounds = true;
+#else
+constexpr bool kCheckBounds = false;
+#endif
+
+// Site ids of the checked accesses.
+enum : uint32_t {
+    kSiteTma = 1, kSiteRowOut = 2, kSiteDrain = 3, kSiteResident = 4, kSiteConst = 5, kSiteZero = 6,
+};
+
+// true when `ok` (always in an unchecked build); otherwise records the site.
+__device__ __forceinline__ bool bound_ok(bool ok, uint32_t *word, uint32_t site) {
+    if constexpr (kCheckBounds) {
+        if (!ok) {
+            if (word) atomicOr(word, kStatusBounds | (site << kStatusSiteShift));
+            return false;
+        }
+    }
+    return true;
+}
+
+// Extent of the tensor behind one TMA map: n0 columns (the head dimension),
+// n1 rows, n2 heads.
+struct MapDims {
+    int n0, n1, n2;
 };
 
 struct DevStatus {
@@ -149,9 +186,17 @@ __device__ __forceinline__ void tc_fence_after() {
 // ---------------------------------------------------------------- TMA
 // 3-D tiled load (coordinates innermost first) into shared memory, completing
 // transaction bytes on `bar`.  The innermost coordinate is always a multiple
-// of 64 elements here, so its byte offset is 16-byte aligned.
+// of 64 elements here, so its byte offset is 16-byte aligned.  `dims` is the
+// map's tensor and `word` the status word, used by the bounds-checked build:
+// the innermost coordinate a multiple of 64 inside the row, the box's first
+// row inside the tensor (later rows past its end are the zero-filled tail),
+// the head in range.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
-                                            int c1, int c2) {
+                                            int c1, int c2, MapDims dims, uint32_t *word) {
+    if (!bound_ok(c0 >= 0 && (c0 & 63) == 0 && c0 + 64 <= dims.n0 && c1 >= 0 && c1 < dims.n1 && c2 >= 0 &&
+                      c2 < dims.n2,
+                  word, kSiteTma))
+        return;
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
@@ -441,17 +486,18 @@ __device__ __forceinline__ void row_to_tmem(uint32_t taddr, const __nv_bfloat16 
 }
 
 // Every one of four warpgroups copies a quarter of the columns of one resident
-// 128-row operand (rows row0 .. row0+127 of head bh of a [BH, N, D] tensor)
-// into tensor memory at column `col`; warp `sub` of a warpgroup must be an
-// SM sub-partition's warp (warp index mod 4), which may touch only lanes
+// 128-row operand (rows row0 .. row0+127 of head bh of a [nheads, N, D]
+// tensor) into tensor memory at column `col`; warp `sub` of a warpgroup must
+// be an SM sub-partition's warp (warp index mod 4), which may touch only lanes
 // 32*sub .. 32*sub+31.
 template <int D>
 __device__ __forceinline__ void resident_to_tmem(uint32_t tmem, uint32_t col, const void *base, int bh, int N, int row0,
-                                                 int wg, int sub, int lane) {
+                                                 int wg, int sub, int lane, int nheads, uint32_t *word) {
     constexpr int W = D / 2 / 4;
     const int r = row0 + sub * 32 + lane;
+    const bool in = r < N && bound_ok(bh >= 0 && bh < nheads && r >= 0 && wg >= 0 && wg < 4, word, kSiteResident);
     const __nv_bfloat16 *src =
-        r < N ? static_cast<const __nv_bfloat16 *>(base) + ((size_t)bh * N + r) * D + wg * 2 * W : nullptr;
+        in ? static_cast<const __nv_bfloat16 *>(base) + ((size_t)bh * N + r) * D + wg * 2 * W : nullptr;
     row_to_tmem<W>(tmem + ((uint32_t)(sub * 32) << 16) + col + wg * W, src);
 }
 

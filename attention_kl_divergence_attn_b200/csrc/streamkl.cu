@@ -492,6 +492,7 @@ const char *streamkl_strerror(streamkl_status s) {
         case STREAMKL_ERR_CUDA: return "CUDA error";
         case STREAMKL_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
         case STREAMKL_ERR_WORKSPACE: return "workspace missing or too small";
+        case STREAMKL_ERR_BOUNDS: return "an access outside its tensor was skipped (bounds-checked build)";
     }
     return "unknown status";
 }
@@ -517,6 +518,7 @@ streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int
     if (code_out) *code_out = word;
     if (cudaPeekAtLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
     if (word & kStatusTimeout) return STREAMKL_ERR_TIMEOUT;
+    if (word & kStatusBounds) return STREAMKL_ERR_BOUNDS;
     return (word & kStatusBadLength) ? STREAMKL_ERR_INVALID_ARG : STREAMKL_OK;
 }
 

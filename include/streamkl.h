@@ -64,7 +64,8 @@ typedef enum {
     STREAMKL_ERR_UNSUPPORTED = 2,   /* valid problem the kernels do not cover (d not 64/128, no sm_100 device) */
     STREAMKL_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
     STREAMKL_ERR_TIMEOUT = 4,       /* a kernel gave up on a bounded wait (see streamkl_check) */
-    STREAMKL_ERR_WORKSPACE = 5      /* workspace NULL or smaller than streamkl_workspace_size() */
+    STREAMKL_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than streamkl_workspace_size() */
+    STREAMKL_ERR_BOUNDS = 6         /* bounds-checked build only: a kernel skipped an access outside its tensor */
 } streamkl_status;
 
 /* Bytes of device workspace that let streamkl_fwd and streamkl_bwd run this
@@ -174,9 +175,12 @@ streamkl_status streamkl_workspace_init(void *workspace, size_t workspace_bytes,
  * earlier call on this workspace gave up on a bounded wait,
  * STREAMKL_ERR_INVALID_ARG if a kernel met a per-batch key length outside
  * [0, N_K] (streamkl_fwd_ex / streamkl_bwd_ex; the length was clamped),
- * STREAMKL_ERR_CUDA if the stream reports a CUDA error, else STREAMKL_OK.
- * `code_out` (host pointer, nullable) receives the raw device status word
- * (0 = clean; bit 0 timeout, bit 1 bad length, bits 8..15 which wait). */
+ * STREAMKL_ERR_BOUNDS if (in the bounds-checked build, libstreamkl_checked.so)
+ * a kernel found a TMA coordinate or global index outside its tensor and
+ * skipped the access, STREAMKL_ERR_CUDA if the stream reports a CUDA error,
+ * else STREAMKL_OK.  `code_out` (host pointer, nullable) receives the raw
+ * device status word (0 = clean; bit 0 timeout, bit 1 bad length, bit 2
+ * bounds, bits 8..15 which wait, bits 16..23 which checked access). */
 streamkl_status streamkl_check(const void *workspace, void *stream, unsigned int *code_out);
 
 /*

@@ -38,8 +38,9 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strerror(L):
     assert L.streamkl_version() >= 100
-    for code in range(6):
+    for code in range(7):
         assert L.streamkl_strerror(code)
+    assert b"unknown" not in L.streamkl_strerror(6)
     assert L.streamkl_workspace_size(1, 1, 128, 128, 64, 64, 0) >= 4
 
 
