@@ -742,16 +742,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     }
 }
 
-// Item r of a persistent CTA: items (head, row tile) are numbered heaviest
-// first and dealt out in rounds of gridDim.x, alternately left to right and
-// right to left, so that every CTA gets a similar share of heavy and light
-// items; -1 once this CTA has none left.
-__device__ __forceinline__ int persistent_item(int r, int n_items) {
-    const long long base = (long long)r * gridDim.x;
-    const long long j = base + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
-    return j < n_items ? (int)j : -1;
-}
-
 template <int DT, int DS, bool TEACHER>
 __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     streamkl_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,

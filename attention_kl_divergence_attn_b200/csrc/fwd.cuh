@@ -480,6 +480,301 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     }
 }
 
+// Persistent form of streamkl_fwd_kernel: one CTA per SM works through its
+// items (one 128-row query tile of one head, or one key split of it; see
+// persistent_item) one after the other.  Key tiles are counted across items,
+// so the K ring, the three logit buffers and their barrier phases simply
+// continue from one item to the next, and tile g goes to the softmax parity
+// g & 1 as in the one-item kernel.  The next item's query rows land in the
+// shared-memory landing area by TMA as soon as the softmax warps have copied
+// the current item's rows into tensor memory, and its first key tiles load
+// while the current item is computed; what remains at an item boundary is the
+// merge of the four warpgroups' row states and the copy of the next rows into
+// tensor memory once the current item's last logit MMA has completed.  Set-up,
+// tensor-memory allocation, the launch and the query-tile load are paid once
+// per SM instead of once per query tile.
+template <int DT, int DS, int NWG>
+__global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
+    streamkl_fwd_persistent_kernel(const __grid_constant__ CUtensorMap mQt, const __grid_constant__ CUtensorMap mKt,
+                                   const __grid_constant__ CUtensorMap mQs, const __grid_constant__ CUtensorMap mKs,
+                                   const FwdParams p) {
+    using C = FwdCfg<DT, DS, NWG>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQt = smem;                  // landing area of the query rows
+    uint8_t *sQs = sQt + C::QT_BYTES;
+    uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
+
+    __shared__ uint64_t bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
+    __shared__ uint64_t bar_q;            // the item's query rows have landed
+    __shared__ uint64_t bar_qfree;        // ... and been copied out of the landing area
+    __shared__ uint64_t bar_qtm;          // ... and are in tensor memory
+    __shared__ uint64_t bar_qtmfree;      // the item's last logit MMA has completed
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+    // per-row states of warpgroups 1..NWG-1, double-buffered by item parity
+    __shared__ float merge[2][NWG > 1 ? NWG - 1 : 1][5][128];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tensors behind the four maps (bounds-checked build)
+    const MapDims mdQt{DT, p.N_Q, p.BH}, mdQs{DS, p.N_Q, p.BH};
+    const MapDims mdKt{DT, p.N_K, p.BH / p.H * p.Hkt}, mdKs{DS, p.N_K, p.BH / p.H * p.Hks};
+    const int off = p.N_K - p.N_Q;
+    const int n_items = p.BH * p.n_qt * p.splits;
+    // item j: as block j of the one-item kernel (heaviest causal tiles first,
+    // the key splits of one query tile adjacent)
+    struct Item {
+        int bh, split, q0, kt_lo, n_kt, bkt, bks;
+    };
+    auto item_geom = [&](int j, bool report) {
+        Item it;
+        const int lin = j / p.BH;
+        it.split = lin % p.splits;
+        it.bh = j % p.BH;
+        it.q0 = (p.n_qt - 1 - lin / p.splits) * C::BM;
+        const int nk = key_count(p.kv_len, it.bh / p.H, p.N_K, p.st.word, report);
+        const int n_all = fwd_key_tiles(it.q0, p.N_Q, nk, off, p.causal, C::BN);
+        it.kt_lo = (int)((long long)n_all * it.split / p.splits);
+        it.n_kt = (int)((long long)n_all * (it.split + 1) / p.splits) - it.kt_lo;
+        it.bkt = key_head(it.bh, p.H, p.Hkt);
+        it.bks = key_head(it.bh, p.H, p.Hks);
+        return it;
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar_q, 1);
+        mbar_init(&bar_qfree, 4 * NWG);   // every softmax warp, once it has copied its rows
+        mbar_init(&bar_qtm, 4 * NWG);     // every softmax warp, once its rows are in tensor memory
+        mbar_init(&bar_qtmfree, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(&bar_kfull[s], 1);
+            mbar_init(&bar_kempty[s], 1);
+        }
+        for (int b = 0; b < C::NBUF; ++b) {
+            mbar_init(&bar_sfull[b], 1);
+            mbar_init(&bar_sempty[b], 4 * C::NH);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+        // the first item's query rows and first key tile right away (the
+        // producer issues the rest after the set-up barrier)
+        prefetch_tmap(&mQt); prefetch_tmap(&mKt); prefetch_tmap(&mQs); prefetch_tmap(&mKs);
+        const Item it = item_geom(persistent_item(0, n_items), true);
+        mbar_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+        for (int b = 0; b < DT / 64; ++b) tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, it.q0, it.bh, mdQt, p.st.word);
+#pragma unroll
+        for (int b = 0; b < DS / 64; ++b) tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, it.q0, it.bh, mdQs, p.st.word);
+        if (it.n_kt > 0) {
+            mbar_expect_tx(&bar_kfull[0], C::STAGE_BYTES);
+#pragma unroll
+            for (int b = 0; b < DT / 64; ++b)
+                tma_load_3d(sK + b * C::KBLK, &mKt, &bar_kfull[0], b * 64, it.kt_lo * C::BN, it.bkt, mdKt, p.st.word);
+#pragma unroll
+            for (int b = 0; b < DS / 64; ++b)
+                tma_load_3d(sK + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[0], b * 64, it.kt_lo * C::BN, it.bks,
+                            mdKs, p.st.word);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int *abort_v = &abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (elect_one()) {
+            int g = 0, issued = 0, q_issued = 1;      // key tiles issued (counted across items), query loads
+            bool ok = true;
+            for (int r = 0, itn = 0; ok; ++r, ++itn) {
+                const int j = persistent_item(r, n_items);
+                if (j < 0) break;
+                const Item it = item_geom(j, false);
+                if (r > 0) {
+                    // the landing area is free once the previous item's rows are copied out
+                    if (!mbar_wait(&bar_qfree, (itn - 1) & 1, p.st, abort_v, 7)) break;
+                    mbar_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b)
+                        tma_load_3d(sQt + b * C::BLK, &mQt, &bar_q, b * 64, it.q0, it.bh, mdQt, p.st.word);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b)
+                        tma_load_3d(sQs + b * C::BLK, &mQs, &bar_q, b * 64, it.q0, it.bh, mdQs, p.st.word);
+                    ++q_issued;
+                }
+                for (int kt = 0; kt < it.n_kt; ++kt, ++g) {
+                    if (r == 0 && kt == 0) {            // issued during set-up
+                        issued = 1;
+                        continue;
+                    }
+                    const int s = g % C::NSTAGE, n = g / C::NSTAGE;
+                    if (n > 0 && !mbar_wait(&bar_kempty[s], (n - 1) & 1, p.st, abort_v, 1)) { ok = false; break; }
+                    uint8_t *st = sK + s * C::STAGE_BYTES;
+                    mbar_expect_tx(&bar_kfull[s], C::STAGE_BYTES);
+#pragma unroll
+                    for (int b = 0; b < DT / 64; ++b)
+                        tma_load_3d(st + b * C::KBLK, &mKt, &bar_kfull[s], b * 64, (it.kt_lo + kt) * C::BN, it.bkt,
+                                    mdKt, p.st.word);
+#pragma unroll
+                    for (int b = 0; b < DS / 64; ++b)
+                        tma_load_3d(st + C::KT_BYTES + b * C::KBLK, &mKs, &bar_kfull[s], b * 64,
+                                    (it.kt_lo + kt) * C::BN, it.bks, mdKs, p.st.word);
+                    issued = g + 1;
+                }
+            }
+            if (*abort_v) {
+                // let copies already in flight land before the CTA's memory is released
+                DevStatus quick = p.st;
+                quick.budget_ns = 50000000ull;
+                volatile int never = 0;
+                mbar_wait(&bar_q, (q_issued - 1) & 1, quick, &never, 1);
+                for (int t = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); t < issued; ++t)
+                    mbar_wait(&bar_kfull[t % C::NSTAGE], (t / C::NSTAGE) & 1, quick, &never, 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);
+        if (elect_one()) {
+            int g = 0;
+            bool ok = true;
+            for (int r = 0, itn = 0; ok; ++r, ++itn) {
+                const int j = persistent_item(r, n_items);
+                if (j < 0) break;
+                const Item it = item_geom(j, false);
+                if (!mbar_wait(&bar_qtm, itn & 1, p.st, abort_v, 2)) break;
+                for (int kt = 0; kt < it.n_kt; ++kt, ++g) {
+                    const int s = g % C::NSTAGE, n = g / C::NSTAGE;
+                    const int buf = g % C::NBUF, use = g / C::NBUF;
+                    if (!mbar_wait(&bar_kfull[s], n & 1, p.st, abort_v, 3)) { ok = false; break; }
+                    if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, p.st, abort_v, 4)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t dKt = desc_add(dK0, s * C::STAGE_BYTES), dKs = desc_add(dKt, C::KT_BYTES);
+                    const uint32_t dSt = tmem + buf * 128, dSs = dSt + 64;
+#pragma unroll
+                    for (int kk = 0; kk < DT / 16; ++kk) {
+                        const uint32_t ok2 = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ts(dSt, tmem + C::TMEM_QT + kk * 8, desc_add(dKt, ok2), C::IDESC, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < DS / 16; ++kk) {
+                        const uint32_t ok2 = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+                        mma_bf16_ts(dSs, tmem + C::TMEM_QS + kk * 8, desc_add(dKs, ok2), C::IDESC, kk > 0);
+                    }
+                    mma_commit(&bar_sfull[buf]);
+                    mma_commit(&bar_kempty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&bar_qtmfree);       // the item's query rows in tensor memory may go
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups (ping-pong)
+        const int wg = (warp - 2) >> 2;
+        const int par = wg & 1, half = wg >> 1;
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        int g0 = 0;
+        for (int r = 0, itn = 0;; ++r, ++itn) {
+            const int j = persistent_item(r, n_items);
+            if (j < 0) break;
+            const Item it = item_geom(j, false);
+            const int grow = it.q0 + row;
+            // this warp's quarter of its 32 rows of Q_t and Q_s into tensor memory,
+            // once they have landed and the previous item's logit MMAs are done.
+            // A wait that gives up ends the item's work but not its merge
+            // barrier, which every softmax warp reaches (the exit is decided there).
+            bool ok = mbar_wait(&bar_q, itn & 1, p.st, abort_v, 6) &&
+                      (itn == 0 || mbar_wait(&bar_qtmfree, (itn - 1) & 1, p.st, abort_v, 8));
+            if (ok) {
+                tc_fence_after();
+                tile_rows_to_tmem<DT>(lane_base + C::TMEM_QT, sQt, wg, row);
+                tile_rows_to_tmem<DS>(lane_base + C::TMEM_QS, sQs, wg, row);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bar_qfree);
+                    mbar_arrive(&bar_qtm);
+                }
+            }
+            float Mt = -INFINITY, Ms = -INFINITY, lt = 0.f, ls = 0.f, A = 0.f;
+            const int nk = key_count(p.kv_len, it.bh / p.H, p.N_K, nullptr, false);
+            for (int kt = 0; ok && kt < it.n_kt; ++kt) {
+                const int g = g0 + kt;
+                if ((g & 1) != par) continue;
+                const int buf = g % C::NBUF;
+                const uint32_t bufc = lane_base + buf * 128;
+                if (!mbar_wait(&bar_sfull[buf], (g / C::NBUF) & 1, p.st, abort_v, 5)) { ok = false; break; }
+                tc_fence_after();
+                const int k0 = (it.kt_lo + kt) * C::BN;
+#pragma unroll
+                for (int cc = 0; cc < C::CW / 32; ++cc) {
+                    const int c = half * (C::CW / 32) + cc;
+                    const int kc = k0 + c * 32;
+                    float ut[32], us[32];
+                    tmem_ld32(bufc + c * 32, ut);
+                    tmem_ld32(bufc + 64 + c * 32, us);
+                    tmem_ld_wait();
+                    const bool masked = (kc + 32 > nk) || (p.causal && (kc + 31 > it.q0 + off));
+                    if (masked) {
+                        const int lim = p.causal ? min(nk, grow + off + 1) : nk;   // first hidden key
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            if (kc + k >= lim) { ut[k] = -INFINITY; us[k] = -INFINITY; }
+                        }
+                        online_chunk_masked(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                    } else {
+                        online_chunk_lag(ut, us, p.ct, p.cs, Mt, Ms, lt, ls, A);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sempty[buf]);
+            }
+            g0 += it.n_kt;
+            // merge the four warpgroups' states (double-buffered by item parity,
+            // so one barrier per item suffices) and write the row outputs; the
+            // barrier also tells every softmax warp alike whether to stop
+            RowState x{Mt, Ms, lt, ls, A};
+            float (*mg)[5][128] = merge[itn & 1];
+            if (wg > 0) {
+                mg[wg - 1][0][row] = Mt; mg[wg - 1][1][row] = Ms; mg[wg - 1][2][row] = lt;
+                mg[wg - 1][3][row] = ls; mg[wg - 1][4][row] = A;
+            }
+            if (bar_sync_or(1, 128 * NWG, !ok || *abort_v)) break;
+            if (wg == 0) {
+#pragma unroll
+                for (int o = 0; o < NWG - 1; ++o)
+                    merge_state(x, RowState{mg[o][0][row], mg[o][1][row], mg[o][2][row], mg[o][3][row], mg[o][4][row]});
+                if (grow < p.N_Q && bound_ok(it.bh < p.BH && it.split < p.splits, p.st.word, kSiteRowOut)) {
+                    const size_t rr = (size_t)it.bh * p.N_Q + grow;
+                    if (p.splits > 1) {
+                        const size_t rows = (size_t)p.BH * p.N_Q, fs = (size_t)p.splits * rows;
+                        float *q = p.part + (size_t)it.split * rows + rr;
+                        q[0] = x.Mt; q[fs] = x.Ms; q[2 * fs] = x.lt; q[3 * fs] = x.ls; q[4 * fs] = x.A;
+                    } else {
+                        finish_row(x, p.kl + rr, p.lse_t + rr, p.lse_s + rr);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
 // Combines the partial states of the key splits of every row, in split
 // order (so the result is the same run to run), and writes the row outputs.
 __global__ void __launch_bounds__(256) streamkl_fwd_merge_kernel(const float *__restrict__ part, int splits,

@@ -77,6 +77,16 @@ __device__ __forceinline__ int key_count(const int *kv_len, int b, int N_K, uint
     return len < 0 ? 0 : (len > N_K ? N_K : len);
 }
 
+// Item r of a persistent CTA: items (head, row tile) are numbered heaviest
+// first and dealt out in rounds of gridDim.x, alternately left to right and
+// right to left, so that every CTA gets a similar share of heavy and light
+// items; -1 once this CTA has none left.
+__device__ __forceinline__ int persistent_item(int r, int n_items) {
+    const long long base = (long long)r * gridDim.x;
+    const long long j = base + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+    return j < n_items ? (int)j : -1;
+}
+
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -181,6 +191,22 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Named barrier `id` over `n` threads (a multiple of 32) that also returns,
+// to every one of them, whether any of them passed `pred` true: a decision
+// all participants take alike.
+__device__ __forceinline__ bool bar_sync_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -162,14 +162,28 @@ size_t dq_split_bytes(int S, long long rows, int d_s, int d_t) {
     return S > 1 ? (size_t)S * rows * (d_s + d_t) * sizeof(float) : 0;
 }
 
+#ifndef STREAMKL_FWD_PERSISTENT
+#define STREAMKL_FWD_PERSISTENT 1
+#endif
+// The forward runs persistent (one CTA per SM working through the query
+// tiles, see streamkl_fwd_persistent_kernel).
+constexpr bool kFwdPersistent = STREAMKL_FWD_PERSISTENT != 0;
+
 template <int DT, int DS>
 streamkl_status launch_fwd(const CUtensorMap &qt, const CUtensorMap &kt, const CUtensorMap &qs,
                            const CUtensorMap &ks, const FwdParams &p, cudaStream_t stream) {
     using C = FwdCfg<DT, DS, kFwdWarpgroups>;
-    auto kern = streamkl_fwd_kernel<DT, DS, kFwdWarpgroups>;
-    if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
-    const long long grid = (long long)p.BH * p.n_qt * p.splits;
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
+    const long long items = (long long)p.BH * p.n_qt * p.splits;
+    if constexpr (kFwdPersistent) {
+        auto kern = streamkl_fwd_persistent_kernel<DT, DS, kFwdWarpgroups>;
+        if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+        const long long grid = std::min<long long>(items, std::max(1, sm_count()));
+        kern<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
+    } else {
+        auto kern = streamkl_fwd_kernel<DT, DS, kFwdWarpgroups>;
+        if (set_smem(kern, C::SMEM) != cudaSuccess) return STREAMKL_ERR_CUDA;
+        kern<<<(unsigned)items, C::THREADS, C::SMEM, stream>>>(qt, kt, qs, ks, p);
+    }
     if (cudaGetLastError() != cudaSuccess) return STREAMKL_ERR_CUDA;
     if (p.splits > 1) {
         const long long rows = (long long)p.BH * p.N_Q;
