@@ -61,13 +61,26 @@ def fwd_flops(w) -> float:
     return 2 * (w.d_t + w.d_s) * visible_pairs(w) * w.B * w.H
 
 
+def key_owner_kernel(w) -> str:
+    """The key-owner kernel the library launches for a workload: the persistent
+    form where the CTA's K rows fit in tensor memory beside the two logit
+    buffers and the dK accumulators (512 columns), else one CTA per key tile."""
+    cols = 256 + w.d_s + (w.d_t if w.teacher_grads else 0) + w.d_t // 2 + w.d_s // 2
+    return "streamkl_bwd_dkv_persistent_kernel" if cols <= 512 else "streamkl_bwd_dkv_kernel"
+
+
+def kernel_names(w) -> list:
+    """The step's kernels in launch order: forward, loss mean, key-owner, query-owner."""
+    return ["streamkl_fwd_persistent_kernel", "streamkl_mean_kernel", key_owner_kernel(w), "streamkl_bwd_dq_kernel"]
+
+
 def kernel_flops(w) -> dict:
     """MMA FLOPs each kernel issues per launch (what its tensor pipe executes)."""
     n = visible_pairs(w) * w.B * w.H
     s = 2 * (w.d_t + w.d_s)                      # S_t and S_s
     g = 2 * w.d_s + (2 * w.d_t if w.teacher_grads else 0)
-    return {"streamkl_fwd_kernel": s * n, "streamkl_bwd_dkv_kernel": (s + g) * n,
-            "streamkl_bwd_dq_kernel": (s + g) * n, "streamkl_mean_kernel": 0.0}
+    fwd, mean, dkv, dq = kernel_names(w)
+    return {fwd: s * n, dkv: (s + g) * n, dq: (s + g) * n, mean: 0.0}
 
 
 def kernel_method_flops(w) -> dict:
@@ -78,8 +91,8 @@ def kernel_method_flops(w) -> dict:
     n = visible_pairs(w) * w.B * w.H
     s = 2 * (w.d_t + w.d_s)
     g = 2 * w.d_s + (2 * w.d_t if w.teacher_grads else 0)
-    return {"streamkl_fwd_kernel": s * n, "streamkl_bwd_dkv_kernel": (s / 2 + g) * n,
-            "streamkl_bwd_dq_kernel": (s / 2 + g) * n, "streamkl_mean_kernel": 0.0}
+    fwd, mean, dkv, dq = kernel_names(w)
+    return {fwd: s * n, dkv: (s / 2 + g) * n, dq: (s / 2 + g) * n, mean: 0.0}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -465,7 +478,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
     kw = dict(stream=stream)
 
-    names = ["streamkl_fwd_kernel", "streamkl_mean_kernel", "streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"]
+    names = kernel_names(w)
 
     outs0 = (kl, lt, ls, loss, dqs, dks, dqt, dkt)
 

@@ -45,7 +45,8 @@ def test_missing_record_gives_no_traffic(tmp_path, monkeypatch):
 def test_committed_record_names_the_step_kernels():
     with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
         rec = json.load(f)
-    assert set(rec["kernels"]) == {"streamkl_fwd_kernel", "streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"}
+    w = inputs.WORKLOADS["causal_8k_d128"]
+    assert set(rec["kernels"]) == {n for n in bench.kernel_names(w) if n != "streamkl_mean_kernel"}
     for e in rec["kernels"].values():
         assert e["workload"] == "causal_8k_d128" and e["dram_bytes_per_launch"] > 0
 
@@ -72,10 +73,19 @@ def test_kernel_method_flops_split_the_step():
     for name in ("causal_8k_d128", "cross_1k_64k", "causal_2k_d64"):
         w = inputs.WORKLOADS[name]
         km, kf = bench.kernel_method_flops(w), bench.kernel_flops(w)
+        fwd, _, dkv, dq = bench.kernel_names(w)
         assert abs(sum(km.values()) - bench.step_flops(w)) <= 1e-9 * bench.step_flops(w)
-        assert km["streamkl_fwd_kernel"] == kf["streamkl_fwd_kernel"]
+        assert km[fwd] == kf[fwd]
         pairs = bench.visible_pairs(w) * w.B * w.H
-        for k in ("streamkl_bwd_dkv_kernel", "streamkl_bwd_dq_kernel"):
+        for k in (dkv, dq):
             assert kf[k] - km[k] == (w.d_t + w.d_s) * pairs
     w = inputs.WORKLOADS["causal_8k_d128"]
     assert bench.kernel_method_flops(w)["streamkl_bwd_dkv_kernel"] == 3 * 256 * bench.visible_pairs(w) * w.H
+
+
+def test_key_owner_form_follows_the_tensor_memory_budget():
+    # the persistent key-owner kernel where the K rows fit in tensor memory
+    # (student-only gradients, or heads of 64): every workload but the 8k one
+    for name, w in inputs.WORKLOADS.items():
+        expect = "streamkl_bwd_dkv_kernel" if name == "causal_8k_d128" else "streamkl_bwd_dkv_persistent_kernel"
+        assert bench.key_owner_kernel(w) == expect, name
