@@ -46,7 +46,10 @@
 // t+2 are issued then, during the dS math of tile t; because MMAs issued by
 // one thread execute in order, the teacher logits of t+2 follow right after
 // the gradient MMA of t, which leaves only half of the next logits on the
-// critical path.
+// critical path.  The two hand-offs of a tile ("student logits read", "dS
+// written") go through named barriers where the resident operand is in
+// shared memory (the d = 128 teacher-and-student forms), and through
+// mbarriers polled by the MMA thread where it is in tensor memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -151,8 +154,9 @@ __device__ __forceinline__ void ds_pair_x2(float ut0, float ut1, float us0, floa
 // values.  The logits are read in pieces of PW columns and each piece's load
 // is issued before the previous piece is computed, so the tensor-memory
 // latency overlaps the arithmetic.  As soon as the last piece has landed the
-// warp arrives on `sfree` (its student logits are no longer needed, so the
-// next tile's student logits may overwrite them); once the whole chunk is
+// warp signals `rel` (an mbarrier, or a named barrier: its student logits are
+// no longer needed, so the next tile's student logits may overwrite them);
+// once the whole chunk is
 // computed, the packed bf16 dS_s (CWID/2 columns) and dS_t (the next CWID/2)
 // are stored over this chunk's teacher logits, which only this warpgroup
 // reads.
@@ -163,6 +167,17 @@ __device__ __forceinline__ void release_student_logits(uint64_t *sfree) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(sfree);
 }
+
+// The same on named barrier `id` (every lane arrives; -1: nobody waits for
+// this tile's release, so no arrival), with n threads taking part.
+struct NamedRel { int id; };
+__device__ __forceinline__ void release_student_logits(NamedRel r, int n) {
+    if (r.id >= 0) {
+        tc_fence_before();
+        named_arrive(r.id, n);
+    }
+}
+__device__ __forceinline__ void release_student_logits(uint64_t *sfree, int) { release_student_logits(sfree); }
 
 template <bool TEACHER, int CWID>
 __device__ __forceinline__ void store_ds(uint32_t at, const uint32_t (&ps)[CWID / 2], const uint32_t (&pt)[CWID / 2]) {
@@ -178,16 +193,16 @@ __device__ __forceinline__ void store_ds(uint32_t at, const uint32_t (&ps)[CWID 
 
 // Query-owner chunk (thread = query row; constants per row, keys kb ..
 // kb+CWID-1, keys >= lim hidden).  The row's g multiplies its dQ at the end.
-template <bool TEACHER, bool MASKED, int CWID, int PW = kBwdPiece>
+template <bool TEACHER, bool MASKED, int CWID, int PW = kBwdPiece, typename Rel>
 __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, float cs, float Lt, float Ls, float g,
-                                         float KL2, int kb, int lim, uint64_t *sfree) {
+                                         float KL2, int kb, int lim, Rel rel, int nsync) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
     uint32_t ps[CWID / 2], pt[CWID / 2];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
     tmem_ld_wait_bind(ut[0], us[0]);
-    if (NP == 1) release_student_logits(sfree);
+    if (NP == 1) release_student_logits(rel, nsync);
 #pragma unroll
     for (int pc = 0; pc < NP; ++pc) {
         const int cur = pc & 1;
@@ -204,7 +219,7 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
-            if (pc + 2 == NP) release_student_logits(sfree);
+            if (pc + 2 == NP) release_student_logits(rel, nsync);
         }
     }
     store_ds<TEACHER, CWID>(at, ps, pt);
@@ -218,9 +233,9 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 // broadcast load per four columns (a quarter of the load instructions of
 // 4-byte loads, for the same shared-memory wavefronts per value; measured
 // 2 % faster).  Columns q < qmin, relative to the chunk, are hidden.
-template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece>
+template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece, typename Rel>
 __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
-                                          const float *gtab, float g_uni, int qmin, uint64_t *sfree) {
+                                          const float *gtab, float g_uni, int qmin, Rel rel, int nsync) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
     float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);   // KL log2(e) of four query columns
@@ -228,7 +243,7 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
     tmem_ld_wait_bind(ut[0], us[0]);
-    if (NP == 1) release_student_logits(sfree);
+    if (NP == 1) release_student_logits(rel, nsync);
 #pragma unroll
     for (int pc = 0; pc < NP; ++pc) {
         const int cur = pc & 1;
@@ -260,7 +275,7 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
-            if (pc + 2 == NP) release_student_logits(sfree);
+            if (pc + 2 == NP) release_student_logits(rel, nsync);
         }
     }
     store_ds<TEACHER, CWID>(at, ps, pt);
@@ -288,6 +303,19 @@ constexpr int kBwdChunk = 64 / kBwdHalves;
 // aligned, as is `ld` * 4 bytes, the row stride.  `lim` is one past the end
 // of the output tensor (checked in the bounds-checked build).
 constexpr int kDrainPad = 4;
+
+// Named barriers of the backward kernels' per-tile hand-off: "dS written"
+// (kNbDsfull + logit buffer) and "student logits read" (kNbSsfree + logit
+// buffer).  The 16 gradient warps arrive (bar.arrive), the whole MMA warp
+// waits (bar.sync): kNbCount threads.  A barrier's next phase cannot start
+// before the MMA warp has passed the current one, because the gradient warps
+// need that tile's logits (committed only after the wait) to reach it.
+// Measured against mbarriers polled by the MMA thread (a per-tile timeline of
+// the query-owner kernel at 8k, d = 128, teacher and student): the MMA thread
+// passed an already completed mbarrier ~240 clk after the last arrival, a
+// named barrier ~35 clk after it.
+constexpr int kNbDsfull = 1, kNbSsfree = 3, kNbCount = 32 * (16 + 1);
+
 
 template <int NCOLS>
 __device__ __forceinline__ void drain_rows(uint32_t taddr, float scale, float *dst, size_t ld, int nvalid,
@@ -414,8 +442,10 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *sOnes = sKs + C::KS_BYTES;            // rank-1 MMA operand (1, 1, 1, 0, ...)
     uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
 
-    __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
-    __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
+    // The per-tile hand-off between the gradient warps and the MMA warp ("dS
+    // written", "student logits read") goes through named barriers kNbDsfull
+    // and kNbSsfree (one per logit buffer).
+    __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2];
     __shared__ uint64_t bar_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -463,8 +493,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&bar_sfull[b], 1);
-                mbar_init(&bar_dsfull[b], 4 * C::NH);
-                mbar_init(&bar_ssfree[b], 4 * C::NH);
             }
             mbar_init(&bar_done, 1);
             abort_flag = 0;
@@ -600,7 +628,9 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dQ0mn = sw128_desc(smem_u32(sQ), C::QBLK, 1024);   // MN-major view of a stage
         const uint64_t dOnes = plain_desc(smem_u32(sOnes), 128, 256);
         const uint64_t dBias0 = plain_desc(smem_u32(sQ + C::BIAS_T), 128, 256);
-        if (elect_one()) {
+        const bool leader = elect_one();
+        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+        {
             // Student S^T of tile t (plus its rank-1 bias -LSE_s / scale_s) into
             // columns [64, 128) of buffer t & 1, once the tile's Q stage has landed.
             auto issue_ss = [&](int t) -> bool {
@@ -638,36 +668,52 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
                 mma_commit(&bar_sfull[buf]);
             };
-            bool ok = C::K_TMEM || mbar_wait(&bar_k, 0, p.st, abort_v, 14);
-            for (int t = 0; ok && t < 2 && t < n_qt; ++t) {
-                ok = issue_ss(t);
-                if (ok) issue_st(t);
+            bool ok = true;
+            if (leader) {
+                ok = C::K_TMEM || mbar_wait(&bar_k, 0, p.st, abort_v, 14);
+                for (int t = 0; ok && t < 2 && t < n_qt; ++t) {
+                    ok = issue_ss(t);
+                    if (ok) issue_st(t);
+                }
             }
-            for (int t = 0; ok && t < n_qt; ++t) {
+            ok = __shfl_sync(0xffffffffu, ok, leader_lane);
+            // The whole warp takes part in the named barriers; after a failed
+            // wait it keeps taking part (issuing nothing), so that the gradient
+            // warps, which make the same arrivals in any case, never wait on it.
+            for (int t = 0; t < n_qt; ++t) {
                 const int buf = t & 1, s = t % C::NSTAGE;
                 const bool next = t + 2 < n_qt;
                 // The student logits of tile t+2 go into this buffer as soon as every
                 // warp has read tile t's (they keep their dS in the teacher half).
-                if (next && (!mbar_wait(&bar_ssfree[buf], (t >> 1) & 1, p.st, abort_v, 13) || !issue_ss(t + 2)))
-                    break;
-                if (!mbar_wait(&bar_dsfull[buf], (t >> 1) & 1, p.st, abort_v, 15)) break;
-                tc_fence_after();
-                const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
-                // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
-#pragma unroll
-                for (int ks = 0; ks < C::BM / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col_s(ks), desc_add(mQs, ks * 2048), C::IDESC_KS,
-                                (t > 0 || ks > 0));
-                if (TEACHER) {
+                __syncwarp();
+                if (next) named_sync(kNbSsfree + buf, kNbCount);
+                if (ok && next) {
+                    tc_fence_after();
+                    bool r = true;
+                    if (leader) r = issue_ss(t + 2);
+                    ok = __shfl_sync(0xffffffffu, r, leader_lane);
+                }
+                named_sync(kNbDsfull + buf, kNbCount);
+                if (ok && leader) {
+                    tc_fence_after();
+                    const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
+                    // dK_s += dS_s^T Q_s : A = dS_s^T from TMEM (buffer columns [0,32)), B = Q_s (MN-major)
 #pragma unroll
                     for (int ks = 0; ks < C::BM / 16; ++ks)
-                        mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + ds_col_t(ks), desc_add(mQt, ks * 2048),
-                                    C::IDESC_KT, (t > 0 || ks > 0));
+                        mma_bf16_ts(tmem + C::TMEM_DKS, tmem + buf * 128 + ds_col_s(ks), desc_add(mQs, ks * 2048),
+                                    C::IDESC_KS, (t > 0 || ks > 0));
+                    if (TEACHER) {
+#pragma unroll
+                        for (int ks = 0; ks < C::BM / 16; ++ks)
+                            mma_bf16_ts(tmem + C::TMEM_DKT, tmem + buf * 128 + ds_col_t(ks), desc_add(mQt, ks * 2048),
+                                        C::IDESC_KT, (t > 0 || ks > 0));
+                    }
+                    mma_commit(&bar_qempty[s]);
+                    if (next) issue_st(t + 2);
                 }
-                mma_commit(&bar_qempty[s]);
-                if (next) issue_st(t + 2);
+                __syncwarp();
             }
-            mma_commit(&bar_done);
+            if (ok && leader) mma_commit(&bar_done);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = key)
@@ -679,33 +725,45 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         constexpr int CW = C::CW;
         const float g_uni = uniform_g(p);
+        static_assert(kBwdParities == 1 && C::THREADS == 32 + kNbCount,
+                      "every gradient warp takes part in every tile's named barriers");
         bool ok = true;
         for (int t = par; t < n_qt; t += kBwdParities) {
             const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
             const int q0 = (first_qt + t) * C::BM;
-            if (!mbar_wait(&bar_sfull[buf], (t >> 1) & 1, p.st, abort_v, 16) ||
-                !mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17)) { ok = false; break; }
+            const int ssid = t + 2 < n_qt ? kNbSsfree + buf : -1;   // the MMA warp waits only when it has a tile t+2
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[buf], (t >> 1) & 1, p.st, abort_v, 16) &&
+                                                 mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17));
+            if (!ok) {
+                // The barriers the MMA warp waits on, without the work.  These
+                // wait too (bar.sync), so that a warp here cannot run ahead into
+                // a later phase of a barrier the MMA warp has not passed.
+                if (ssid >= 0) named_sync(ssid, kNbCount);
+                named_sync(kNbDsfull + buf, kNbCount);
+                continue;
+            }
             tc_fence_after();
             const float *ktab = reinterpret_cast<const float *>(sQ + s * C::STAGE_BYTES + C::GK) + half * CW;
             const float *gtab = ktab + C::BM;
             const int qmin = gk - off - q0;        // first visible query column (causal)
             const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
             const bool masked = p.causal && (k0 + C::BN - 1 > q0 + half * CW + off);
-            uint64_t *sfree = &bar_ssfree[buf];
+            const NamedRel rel{ssid};
             if (masked) {
                 if (p.dkl)
-                    dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW, sfree);
+                    dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW, rel,
+                                                       kNbCount);
                 else
-                    dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW,
-                                                        sfree);
+                    dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW, rel,
+                                                        kNbCount);
             } else {
-                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, sfree);
-                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, sfree);
+                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, rel, kNbCount);
+                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, rel, kNbCount);
             }
             tmem_st_wait();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
+            named_arrive(kNbDsfull + buf, kNbCount);
         }
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
@@ -1196,13 +1254,13 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     if (masked) {
                         if (p.dkl)
                             dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f,
-                                                               qmin - half * CW, sfree);
+                                                               qmin - half * CW, sfree, 0);
                         else
                             dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni,
-                                                                qmin - half * CW, sfree);
+                                                                qmin - half * CW, sfree, 0);
                     } else {
-                        if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, sfree);
-                        else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, sfree);
+                        if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, sfree, 0);
+                        else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, sfree, 0);
                     }
                     tmem_st_wait();
                     tc_fence_before();
@@ -1266,6 +1324,11 @@ struct DqCfg {
     static constexpr uint32_t TMEM_DQS = 256, TMEM_DQT = 256 + DS;
     static constexpr uint32_t TMEM_QT = TMEM_DQT + (TEACHER ? DT : 0), TMEM_QS = TMEM_QT + DT / 2;
     static constexpr bool Q_TMEM = TMEM_QS + DS / 2 <= 512;
+    // Hand-off of each tile between the gradient warps and the MMA warp through
+    // named barriers where the logit MMAs read Q from shared memory; through
+    // mbarriers (polled by the MMA thread) where Q sits in tensor memory, the
+    // form in which the named barriers measured slower.
+    static constexpr bool NAMED = !Q_TMEM;
     static constexpr int QT_BYTES = Q_TMEM ? 0 : BM * DT * 2, QS_BYTES = Q_TMEM ? 0 : BM * DS * 2;
     static constexpr int KT_BYTES = BN * DT * 2, KS_BYTES = BN * DS * 2;
     static constexpr int STAGE_BYTES = KT_BYTES + KS_BYTES;
@@ -1416,7 +1479,9 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dQt = sw128_desc(smem_u32(sQt), 16, 1024), dQs = sw128_desc(smem_u32(sQs), 16, 1024);
         const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);          // K-major view of a stage
         const uint64_t dK0mn = sw128_desc(smem_u32(sK), C::KBLK, 1024);   // MN-major view of a stage
-        if (elect_one()) {
+        const bool leader = elect_one();
+        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+        {
             // Student S of key tile kt into columns [64, 128) of buffer kt & 1,
             // once the tile's K stage has landed.
             auto issue_ss = [&](int kt) -> bool {
@@ -1450,26 +1515,15 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 }
                 mma_commit(&bar_sfull[buf]);
             };
-            bool ok = C::Q_TMEM || mbar_wait(&bar_q, 0, p.st, abort_v, 24);
-            for (int kt = 0; ok && kt < 2 && kt < n_kt; ++kt) {
-                ok = issue_ss(kt);
-                if (ok) issue_st(kt);
-            }
-            for (int kt = 0; ok && kt < n_kt; ++kt) {
-                const int buf = kt & 1, s = kt % C::NSTAGE;
-                const bool next = kt + 2 < n_kt;
-                // the student logits of tile kt+2 go into this buffer as soon as
-                // every warp has read tile kt's (they keep their dS in the teacher half)
-                if (next && (!mbar_wait(&bar_ssfree[buf], (kt >> 1) & 1, p.st, abort_v, 23) || !issue_ss(kt + 2)))
-                    break;
-                if (!mbar_wait(&bar_dsfull[buf], (kt >> 1) & 1, p.st, abort_v, 25)) break;
-                tc_fence_after();
+            // dQ += dS K for tile kt (A = dS from TMEM, buffer columns [0, 32) for
+            // the student, B = the K stage, MN-major), then release the stage.
+            auto issue_dq = [&](int kt) {
+                const int s = kt % C::NSTAGE, buf = kt & 1;
                 const uint64_t mKt = desc_add(dK0mn, s * C::STAGE_BYTES), mKs = desc_add(mKt, C::KT_BYTES);
-                // dQ_s += dS_s K_s : A = dS_s from TMEM (buffer columns [0,32)), B = K_s (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks)
-                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col_s(ks), desc_add(mKs, ks * 2048), C::IDESC_QS,
-                                (kt > 0 || ks > 0));
+                    mma_bf16_ts(tmem + C::TMEM_DQS, tmem + buf * 128 + ds_col_s(ks), desc_add(mKs, ks * 2048),
+                                C::IDESC_QS, (kt > 0 || ks > 0));
                 if (TEACHER) {
 #pragma unroll
                     for (int ks = 0; ks < C::BN / 16; ++ks)
@@ -1477,9 +1531,55 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                                     C::IDESC_QT, (kt > 0 || ks > 0));
                 }
                 mma_commit(&bar_kempty[s]);
-                if (next) issue_st(kt + 2);
+            };
+            bool ok = true;
+            if (leader) {
+                ok = C::Q_TMEM || mbar_wait(&bar_q, 0, p.st, abort_v, 24);
+                for (int kt = 0; ok && kt < 2 && kt < n_kt; ++kt) {
+                    ok = issue_ss(kt);
+                    if (ok) issue_st(kt);
+                }
             }
-            mma_commit(&bar_done);
+            if constexpr (C::NAMED) {
+                ok = __shfl_sync(0xffffffffu, ok, leader_lane);
+                // The whole warp takes part in the named barriers; after a failed
+                // wait it keeps taking part (issuing nothing), so that the gradient
+                // warps, which make the same arrivals in any case, never wait on it.
+                for (int kt = 0; kt < n_kt; ++kt) {
+                    const int buf = kt & 1;
+                    const bool next = kt + 2 < n_kt;
+                    // the student logits of tile kt+2 go into this buffer as soon as
+                    // every warp has read tile kt's (they keep their dS in the teacher half)
+                    __syncwarp();
+                    if (next) named_sync(kNbSsfree + buf, kNbCount);
+                    if (ok && next) {
+                        tc_fence_after();
+                        bool r = true;
+                        if (leader) r = issue_ss(kt + 2);
+                        ok = __shfl_sync(0xffffffffu, r, leader_lane);
+                    }
+                    named_sync(kNbDsfull + buf, kNbCount);
+                    if (ok && leader) {
+                        tc_fence_after();
+                        issue_dq(kt);
+                        if (next) issue_st(kt + 2);
+                    }
+                    __syncwarp();
+                }
+                if (ok && leader) mma_commit(&bar_done);
+            } else if (leader) {
+                for (int kt = 0; ok && kt < n_kt; ++kt) {
+                    const int buf = kt & 1;
+                    const bool next = kt + 2 < n_kt;
+                    if (next && (!mbar_wait(&bar_ssfree[buf], (kt >> 1) & 1, p.st, abort_v, 23) || !issue_ss(kt + 2)))
+                        break;
+                    if (!mbar_wait(&bar_dsfull[buf], (kt >> 1) & 1, p.st, abort_v, 25)) break;
+                    tc_fence_after();
+                    issue_dq(kt);
+                    if (next) issue_st(kt + 2);
+                }
+                mma_commit(&bar_done);
+            }
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = query)
@@ -1498,22 +1598,45 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             KL2 = p.kl[r] * kLog2eF;
         }
         const int lim = p.causal ? min(nk, gq + off + 1) : nk;   // first hidden key
+        static_assert(kBwdParities == 1 && C::THREADS == 32 + kNbCount,
+                      "every gradient warp takes part in every tile's hand-off");
         bool ok = true;
         for (int kt = par; kt < n_kt; kt += kBwdParities) {
             const int buf = kt & 1;
-            if (!mbar_wait(&bar_sfull[buf], (kt >> 1) & 1, p.st, abort_v, 26)) { ok = false; break; }
+            const int ssid = kt + 2 < n_kt ? kNbSsfree + buf : -1;   // the MMA warp waits only when it has a tile t+2
+            if constexpr (C::NAMED) {
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[buf], (kt >> 1) & 1, p.st, abort_v, 26));
+                if (!ok) {
+                    // The barriers the MMA warp waits on, without the work.  These
+                    // wait too (bar.sync), so that a warp here cannot run ahead into
+                    // a later phase of a barrier the MMA warp has not passed.
+                    if (ssid >= 0) named_sync(ssid, kNbCount);
+                    named_sync(kNbDsfull + buf, kNbCount);
+                    continue;
+                }
+            } else {
+                if (!mbar_wait(&bar_sfull[buf], (kt >> 1) & 1, p.st, abort_v, 26)) { ok = false; break; }
+            }
             tc_fence_after();
+            const auto rel = [&] {
+                if constexpr (C::NAMED) return NamedRel{ssid};
+                else return &bar_ssfree[buf];
+            }();
             const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
             const int kb = (kt_lo + kt) * C::BN + half * CW;
             const bool masked = (kb + CW > nk) || (p.causal && (kb + CW - 1 > q0 + off));
             if (masked)
-                dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, &bar_ssfree[buf]);
+                dq_chunk<TEACHER, true, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, rel, kNbCount);
             else
-                dq_chunk<TEACHER, false, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, &bar_ssfree[buf]);
+                dq_chunk<TEACHER, false, CW>(col, col + 64, p.ct, p.cs, Lt, Ls, g, KL2, kb, lim, rel, kNbCount);
             tmem_st_wait();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
+            if constexpr (C::NAMED) {
+                named_arrive(kNbDsfull + buf, kNbCount);
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
+            }
         }
         if (ok && mbar_wait(&bar_done, 0, p.st, abort_v, 28)) {
             tc_fence_after();

@@ -196,6 +196,15 @@ __device__ __forceinline__ void tc_fence_after() {
 // Named barrier `id` over `n` threads (a multiple of 32) that also returns,
 // to every one of them, whether any of them passed `pred` true: a decision
 // all participants take alike.
+// Named CTA barriers (bar.sync / bar.arrive, aligned: every lane of a warp
+// executes them; n counts threads, a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ bool bar_sync_or(int id, int n, bool pred) {
     uint32_t r;
     asm volatile(
