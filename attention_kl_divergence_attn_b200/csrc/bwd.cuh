@@ -447,6 +447,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     // and kNbSsfree (one per logit buffer).
     __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2];
     __shared__ uint64_t bar_done;
+    __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -495,6 +496,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 mbar_init(&bar_sfull[b], 1);
             }
             mbar_init(&bar_done, 1);
+            mbar_init(&bar_quiet, 1);
             abort_flag = 0;
             fence_barrier_init();
             if (!C::K_TMEM) {
@@ -714,6 +716,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 __syncwarp();
             }
             if (ok && leader) mma_commit(&bar_done);
+            if (leader) mma_quiesce(&bar_quiet, p.st, 29);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = key)
@@ -829,6 +832,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ uint64_t bar_k;                     // this item's resident K rows are in place
     __shared__ uint64_t bar_kfree;                 // the item's last logit MMA has completed
     __shared__ uint64_t bar_done;                  // the item's last gradient MMA has completed
+    __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
     __shared__ uint64_t bar_kst, bar_kstfree;      // K_TMEM: staged K rows landed / copied out
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -865,6 +869,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             mbar_init(&bar_k, C::K_TMEM ? 4 * C::NH : 1);
             mbar_init(&bar_kfree, 1);
             mbar_init(&bar_done, 1);
+            mbar_init(&bar_quiet, 1);
             mbar_init(&bar_kst, 1);
             mbar_init(&bar_kstfree, 4 * C::NH);
             abort_flag = 0;
@@ -1184,6 +1189,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 g0 += n_qt;
                 ++it;
             }
+            mma_quiesce(&bar_quiet, p.st, 29);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = key)
@@ -1362,6 +1368,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
     __shared__ uint64_t bar_q, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[2], bar_dsfull[2];
     __shared__ uint64_t bar_ssfree[2];             // all warps have read the buffer's student logits
     __shared__ uint64_t bar_done;
+    __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -1399,6 +1406,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             mbar_init(&bar_ssfree[b], 4 * C::NH);
         }
         mbar_init(&bar_done, 1);
+        mbar_init(&bar_quiet, 1);
         abort_flag = 0;
         fence_barrier_init();
         // Start the resident Q tile and the first K stage right away, so that
@@ -1580,6 +1588,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 }
                 mma_commit(&bar_done);
             }
+            if (leader) mma_quiesce(&bar_quiet, p.st, 29);
         }
     } else {
         // ------------------------------------------------------------ gradient warpgroups (thread = query)

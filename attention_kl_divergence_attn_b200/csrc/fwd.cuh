@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
 
     __shared__ uint64_t bar_q, bar_qtm, bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
+    __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ float merge[NWG > 1 ? NWG - 1 : 1][5][128];   // per-row states of warpgroups 1..NWG-1
@@ -305,6 +306,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             mbar_init(&bar_sfull[b], 1);
             mbar_init(&bar_sempty[b], 4 * C::NH);
         }
+        mbar_init(&bar_quiet, 1);
         abort_flag = 0;
         fence_barrier_init();
         // Start the query tile and the first K stage right away, so that their
@@ -396,6 +398,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                     mma_commit(&bar_kempty[s]);
                 }
             }
+            mma_quiesce(&bar_quiet, p.st, 9);
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups (ping-pong)
@@ -506,6 +509,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
     uint8_t *sK = sQs + C::QS_BYTES;      // stage s: K_t then K_s
 
     __shared__ uint64_t bar_kfull[C::NSTAGE], bar_kempty[C::NSTAGE], bar_sfull[C::NBUF], bar_sempty[C::NBUF];
+    __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
     __shared__ uint64_t bar_q;            // the item's query rows have landed
     __shared__ uint64_t bar_qfree;        // ... and been copied out of the landing area
     __shared__ uint64_t bar_qtm;          // ... and are in tensor memory
@@ -554,6 +558,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
             mbar_init(&bar_sfull[b], 1);
             mbar_init(&bar_sempty[b], 4 * C::NH);
         }
+        mbar_init(&bar_quiet, 1);
         abort_flag = 0;
         fence_barrier_init();
         // the first item's query rows and first key tile right away (the
@@ -672,6 +677,7 @@ __global__ void __launch_bounds__(FwdCfg<DT, DS, NWG>::THREADS, 1)
                 if (!ok) break;
                 mma_commit(&bar_qtmfree);       // the item's query rows in tensor memory may go
             }
+            mma_quiesce(&bar_quiet, p.st, 9);
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups (ping-pong)

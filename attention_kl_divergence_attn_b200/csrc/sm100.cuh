@@ -289,6 +289,19 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  : "memory");
 }
 
+// Before a CTA frees its tensor memory, every MMA that this thread issued must
+// have completed.  On the normal path they have (their results were read);
+// on a path that gave up early some may still be running.  The thread
+// commits to `bar` (an mbarrier for this one use, one arrival) and waits for
+// it with a short bounded wait of its own.
+__device__ __forceinline__ void mma_quiesce(uint64_t *bar, const DevStatus &st, uint32_t who) {
+    mma_commit(bar);
+    DevStatus quick = st;
+    quick.budget_ns = 50000000ull;
+    volatile int never = 0;
+    mbar_wait(bar, 0, quick, &never, who);
+}
+
 // 32 lanes x 32 consecutive fp32 columns: thread t of the warp gets lane
 // (warp's lane quarter base + t), columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
