@@ -304,17 +304,27 @@ constexpr int kBwdChunk = 64 / kBwdHalves;
 // of the output tensor (checked in the bounds-checked build).
 constexpr int kDrainPad = 4;
 
-// Named barriers of the backward kernels' per-tile hand-off: "dS written"
-// (kNbDsfull + logit buffer) and "student logits read" (kNbSsfree + logit
-// buffer).  The 16 gradient warps arrive (bar.arrive), the whole MMA warp
-// waits (bar.sync): kNbCount threads.  A barrier's next phase cannot start
-// before the MMA warp has passed the current one, because the gradient warps
-// need that tile's logits (committed only after the wait) to reach it.
-// Measured against mbarriers polled by the MMA thread (a per-tile timeline of
-// the query-owner kernel at 8k, d = 128, teacher and student): the MMA thread
-// passed an already completed mbarrier ~240 clk after the last arrival, a
-// named barrier ~35 clk after it.
-constexpr int kNbDsfull = 1, kNbSsfree = 3, kNbCount = 32 * (16 + 1);
+// Named barriers of the backward kernels' per-tile hand-off: "dS written" of
+// tile t on id nb_dsfull(t) and "student logits read" on nb_ssfree(t), four
+// ids of each kind used in turn.  The 16 gradient warps arrive (bar.arrive),
+// the whole MMA warp waits (bar.sync): kNbCount threads.  A gradient warp's
+// arrivals run at most two tiles ahead of the MMA warp's waits (tile t's
+// logits are committed only after the MMA warp has passed tile t-2), so
+// while their logits come, no id is reused before its phase has completed.
+// A warp whose bounded wait gave up no longer waits for logits; it takes part
+// in each remaining tile's barriers with bar.sync, which cannot complete
+// before the MMA warp's wait on the same tile, so from its first such tile on
+// it stays in step.  With one id per logit buffer that first tile (t+2 after
+// its last arrival for t) would share the id of a phase still open: the
+// phase would complete with the arrivals of two tiles and the MMA warp's
+// later wait never (tests/test_handoff_protocol.py runs the protocol as a
+// model).  Measured against mbarriers polled by the MMA thread (a per-tile
+// timeline of the query-owner kernel at 8k, d = 128, teacher and student):
+// the MMA thread passed an already completed mbarrier ~240 clk after the last
+// arrival, a named barrier ~35 clk after it.
+constexpr int kNbDsfullBase = 1, kNbSsfreeBase = 5, kNbCount = 32 * (16 + 1);
+__host__ __device__ constexpr int nb_dsfull(int t) { return kNbDsfullBase + (t & 3); }
+__host__ __device__ constexpr int nb_ssfree(int t) { return kNbSsfreeBase + (t & 3); }
 
 
 template <int NCOLS>
@@ -443,8 +453,8 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
 
     // The per-tile hand-off between the gradient warps and the MMA warp ("dS
-    // written", "student logits read") goes through named barriers kNbDsfull
-    // and kNbSsfree (one per logit buffer).
+    // written", "student logits read") goes through named barriers
+    // nb_dsfull(t) and nb_ssfree(t).
     __shared__ uint64_t bar_k, bar_qfull[C::NSTAGE], bar_qempty[C::NSTAGE], bar_sfull[2];
     __shared__ uint64_t bar_done;
     __shared__ uint64_t bar_quiet;                 // the MMA thread's issued MMAs have completed
@@ -688,14 +698,14 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 // The student logits of tile t+2 go into this buffer as soon as every
                 // warp has read tile t's (they keep their dS in the teacher half).
                 __syncwarp();
-                if (next) named_sync(kNbSsfree + buf, kNbCount);
+                if (next) named_sync(nb_ssfree(t), kNbCount);
                 if (ok && next) {
                     tc_fence_after();
                     bool r = true;
                     if (leader) r = issue_ss(t + 2);
                     ok = __shfl_sync(0xffffffffu, r, leader_lane);
                 }
-                named_sync(kNbDsfull + buf, kNbCount);
+                named_sync(nb_dsfull(t), kNbCount);
                 if (ok && leader) {
                     tc_fence_after();
                     const uint64_t mQt = desc_add(dQ0mn, s * C::STAGE_BYTES), mQs = desc_add(mQt, C::QT_BYTES);
@@ -734,16 +744,16 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         for (int t = par; t < n_qt; t += kBwdParities) {
             const int s = t % C::NSTAGE, n = t / C::NSTAGE, buf = t & 1;
             const int q0 = (first_qt + t) * C::BM;
-            const int ssid = t + 2 < n_qt ? kNbSsfree + buf : -1;   // the MMA warp waits only when it has a tile t+2
+            const int ssid = t + 2 < n_qt ? nb_ssfree(t) : -1;   // the MMA warp waits only when it has a tile t+2
             if (ok)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[buf], (t >> 1) & 1, p.st, abort_v, 16) &&
                                                  mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 17));
             if (!ok) {
                 // The barriers the MMA warp waits on, without the work.  These
-                // wait too (bar.sync), so that a warp here cannot run ahead into
-                // a later phase of a barrier the MMA warp has not passed.
+                // wait too (bar.sync), so that a warp here stays in step with the
+                // MMA warp (the ids go round four tiles: see nb_dsfull).
                 if (ssid >= 0) named_sync(ssid, kNbCount);
-                named_sync(kNbDsfull + buf, kNbCount);
+                named_sync(nb_dsfull(t), kNbCount);
                 continue;
             }
             tc_fence_after();
@@ -766,7 +776,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            named_arrive(kNbDsfull + buf, kNbCount);
+            named_arrive(nb_dsfull(t), kNbCount);
         }
         if (ok && n_qt > 0 && mbar_wait(&bar_done, 0, p.st, abort_v, 19)) {
             tc_fence_after();
@@ -1559,14 +1569,14 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                     // the student logits of tile kt+2 go into this buffer as soon as
                     // every warp has read tile kt's (they keep their dS in the teacher half)
                     __syncwarp();
-                    if (next) named_sync(kNbSsfree + buf, kNbCount);
+                    if (next) named_sync(nb_ssfree(kt), kNbCount);
                     if (ok && next) {
                         tc_fence_after();
                         bool r = true;
                         if (leader) r = issue_ss(kt + 2);
                         ok = __shfl_sync(0xffffffffu, r, leader_lane);
                     }
-                    named_sync(kNbDsfull + buf, kNbCount);
+                    named_sync(nb_dsfull(kt), kNbCount);
                     if (ok && leader) {
                         tc_fence_after();
                         issue_dq(kt);
@@ -1612,15 +1622,15 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
         bool ok = true;
         for (int kt = par; kt < n_kt; kt += kBwdParities) {
             const int buf = kt & 1;
-            const int ssid = kt + 2 < n_kt ? kNbSsfree + buf : -1;   // the MMA warp waits only when it has a tile t+2
+            const int ssid = kt + 2 < n_kt ? nb_ssfree(kt) : -1;   // the MMA warp waits only when it has a tile t+2
             if constexpr (C::NAMED) {
                 if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[buf], (kt >> 1) & 1, p.st, abort_v, 26));
                 if (!ok) {
                     // The barriers the MMA warp waits on, without the work.  These
-                    // wait too (bar.sync), so that a warp here cannot run ahead into
-                    // a later phase of a barrier the MMA warp has not passed.
+                    // wait too (bar.sync), so that a warp here stays in step with the
+                    // MMA warp (the ids go round four tiles: see nb_dsfull).
                     if (ssid >= 0) named_sync(ssid, kNbCount);
-                    named_sync(kNbDsfull + buf, kNbCount);
+                    named_sync(nb_dsfull(kt), kNbCount);
                     continue;
                 }
             } else {
@@ -1641,7 +1651,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
             tmem_st_wait();
             tc_fence_before();
             if constexpr (C::NAMED) {
-                named_arrive(kNbDsfull + buf, kNbCount);
+                named_arrive(nb_dsfull(kt), kNbCount);
             } else {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_dsfull[buf]);
