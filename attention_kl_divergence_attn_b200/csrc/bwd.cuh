@@ -1564,7 +1564,7 @@ __global__ void __launch_bounds__(DqCfg<DT, DS, TEACHER>::THREADS, 1)
                 // wait it keeps taking part (issuing nothing), so that the gradient
                 // warps, which make the same arrivals in any case, never wait on it.
                 for (int kt = 0; kt < n_kt; ++kt) {
-                    const int buf = kt & 1;
+                    // tile kt hands off on nb_ssfree(kt) and nb_dsfull(kt)
                     const bool next = kt + 2 < n_kt;
                     // the student logits of tile kt+2 go into this buffer as soon as
                     // every warp has read tile kt's (they keep their dS in the teacher half)
