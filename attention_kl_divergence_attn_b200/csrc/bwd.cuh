@@ -17,14 +17,15 @@
 // deterministic result):
 //   streamkl_bwd_dkv_kernel  CTA = 128 keys of one head; loops over 64-query
 //       tiles: S^T = K Q^T (teacher and student), dS^T, dK += dS^T Q.
-//       Thread = key row, so the per-query log-sum-exps would be a per-element
-//       shared-memory load; instead one extra rank-1 MMA per tensor and tile
-//       adds them to the logits: A = a constant [128 x 16] matrix whose rows
-//       are (1, 1, 1, 0, ...), B = the tile's rows (h, m, l, 0, ...) with
+//       Thread = key row, so the per-query values (KL, the two log-sum-exps,
+//       and g when it varies per row) come from a small per-stage table in
+//       shared memory, read with one 16-byte broadcast load per four queries.
+//       The persistent form (K in tensor memory), whose gradient warps are its
+//       limit, instead adds the log-sum-exps to the logits with one extra
+//       rank-1 MMA per tensor and tile: A = a constant [128 x 16] matrix whose
+//       rows are (1, 1, 1, 0, ...), B = the tile's rows (h, m, l, 0, ...) with
 //       h + m + l = -LSE / scale split into three bf16 terms (about fp32
 //       precision), so the accumulator holds q.k - LSE / scale directly.
-//       Only KL per query (and g, when it varies per row) comes from a small
-//       shared-memory table, read with one broadcast load per pair of queries.
 //   streamkl_bwd_dq_kernel   CTA = 128 queries of one head; loops over 64-key
 //       tiles: S = Q K^T, dS, dQ += dS K.  Thread = query row; per-row
 //       constants live in registers.
@@ -233,12 +234,15 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
 // broadcast load per four columns (a quarter of the load instructions of
 // 4-byte loads, for the same shared-memory wavefronts per value; measured
 // 2 % faster).  Columns q < qmin, relative to the chunk, are hidden.
-template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece, typename Rel>
+template <bool TEACHER, bool MASKED, bool G_ROW, int CWID, int PW = kBwdPiece, typename Rel, bool LTAB = false>
 __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, float cs, const float *ktab,
-                                          const float *gtab, float g_uni, int qmin, Rel rel, int nsync) {
+                                          const float *gtab, float g_uni, int qmin, Rel rel, int nsync,
+                                          const float *ltab = nullptr, const float *stab = nullptr) {
     constexpr int NP = CWID / PW;
     float ut[2][PW], us[2][PW];
     float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);   // KL log2(e) of four query columns
+    float4 l4 = make_float4(0.f, 0.f, 0.f, 0.f);   // LTAB: -LSE_t log2(e) of the same four columns
+    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);   // LTAB: -LSE_s log2(e)
     uint32_t ps[CWID / 2], pt[CWID / 2];
     tmem_ld<PW>(at, ut[0]);
     tmem_ld<PW>(as, us[0]);
@@ -254,7 +258,7 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
 #pragma unroll
         for (int k = 0; k < PW; k += 2) {
             const int q = PW * pc + k;
-            float2 K = make_float2(0.f, 0.f);
+            float2 K = make_float2(0.f, 0.f), NL = make_float2(0.f, 0.f), NS = make_float2(0.f, 0.f);
             if constexpr (TEACHER) {
                 if ((q & 3) == 0) {
                     k4 = ld_shared_v4(ktab + q);
@@ -263,15 +267,28 @@ __device__ __forceinline__ void dkv_chunk(uint32_t at, uint32_t as, float ct, fl
                     K = make_float2(k4.z, k4.w);
                 }
             }
+            if constexpr (LTAB) {
+                if ((q & 3) == 0) {
+                    l4 = ld_shared_v4(ltab + q);
+                    s4 = ld_shared_v4(stab + q);
+                    NL = make_float2(l4.x, l4.y);
+                    NS = make_float2(s4.x, s4.y);
+                } else {
+                    NL = make_float2(l4.z, l4.w);
+                    NS = make_float2(s4.z, s4.w);
+                }
+            }
             const float2 G = G_ROW ? *reinterpret_cast<const float2 *>(gtab + q) : make_float2(g_uni, g_uni);
             if constexpr (G_ROW)
-                ds_pair<TEACHER, MASKED, true>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs, 0.f, 0.f,
-                                               0.f, 0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin, ps[q >> 1],
-                                               pt[q >> 1]);
+                ds_pair<TEACHER, MASKED, true>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], ct, cs,
+                                               LTAB ? -NL.x : 0.f, LTAB ? -NL.y : 0.f, LTAB ? -NS.x : 0.f,
+                                               LTAB ? -NS.y : 0.f, G.x, G.y, K.x, K.y, q >= qmin, q + 1 >= qmin,
+                                               ps[q >> 1], pt[q >> 1]);
             else
                 ds_pair_x2<TEACHER, MASKED>(ut[cur][k], ut[cur][k + 1], us[cur][k], us[cur][k + 1], f2splat(ct),
-                                            f2splat(cs), 0ull, 0ull, f2pack(K.x, K.y), q >= qmin, q + 1 >= qmin,
-                                            ps[q >> 1], pt[q >> 1]);
+                                            f2splat(cs), LTAB ? f2pack(NL.x, NL.y) : 0ull,
+                                            LTAB ? f2pack(NS.x, NS.y) : 0ull, f2pack(K.x, K.y), q >= qmin,
+                                            q + 1 >= qmin, ps[q >> 1], pt[q >> 1]);
         }
         if (pc + 1 < NP) {
             tmem_ld_wait_bind(ut[cur ^ 1], us[cur ^ 1]);
@@ -407,11 +424,20 @@ struct DkvCfg {
     static constexpr int KT_BYTES = K_TMEM ? 0 : BN * DT * 2, KS_BYTES = K_TMEM ? 0 : BN * DS * 2;
     static constexpr int QT_BYTES = BM * DT * 2, QS_BYTES = BM * DS * 2;
     static constexpr int STAGE_TMA = QT_BYTES + QS_BYTES;
-    static constexpr int BIAS_BYTES = BM * 16 * 2;  // [64 queries][16] bf16, unswizzled K-major
-    static constexpr int GK_BYTES = BM * 8;         // KL log2(e) per query, then g per query
+    // The per-query log-sum-exps reach the logits in one of two ways.
+    // LSE_TAB (the one-item kernel, K in shared memory): from a per-stage table
+    // that the gradient warps read with the KL values (16-byte broadcast
+    // loads), subtracted in their first fused multiply-add.  Otherwise (the
+    // persistent kernel): by one rank-1 bias MMA per tensor and tile.  The
+    // one-item kernel at d = 128 is limited by its MMAs, the persistent one by
+    // its gradient warps, so each takes the work where it has room.
+    static constexpr bool LSE_TAB = !K_TMEM;
+    static constexpr int BIAS_BYTES = LSE_TAB ? 0 : BM * 16 * 2;  // [64 queries][16] bf16, unswizzled K-major
+    // per query: KL log2(e), then g, then (LSE_TAB) -LSE_t log2(e) and -LSE_s log2(e)
+    static constexpr int GK_BYTES = BM * (LSE_TAB ? 16 : 8);
     static constexpr int BIAS_T = STAGE_TMA, BIAS_S = BIAS_T + BIAS_BYTES, GK = BIAS_S + BIAS_BYTES;
     static constexpr int STAGE_BYTES = ((GK + GK_BYTES + 1023) / 1024) * 1024;
-    static constexpr int ONES_BYTES = BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
+    static constexpr int ONES_BYTES = LSE_TAB ? 0 : BN * 16 * 2;  // [128 keys][16] bf16 rows (1, 1, 1, 0, ...)
     // K_STAGED (persistent form, K in tensor memory): the next item's K rows
     // land in a staging area by TMA (K_t boxes, then K_s boxes) and the
     // gradient warps copy them into tensor memory.  Used when the Q ring keeps
@@ -449,8 +475,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sKt = smem;
     uint8_t *sKs = sKt + C::KT_BYTES;
-    uint8_t *sOnes = sKs + C::KS_BYTES;            // rank-1 MMA operand (1, 1, 1, 0, ...)
-    uint8_t *sQ = sOnes + C::ONES_BYTES;           // stages: Q_t, Q_s, bias_t, bias_s, {g, KL}
+    uint8_t *sQ = sKs + C::KS_BYTES;               // stages: Q_t, Q_s, then per query {KL, g, -LSE_t, -LSE_s}
 
     // The per-tile hand-off between the gradient warps and the MMA warp ("dS
     // written", "student logits read") goes through named barriers
@@ -532,24 +557,7 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         tmem_alloc(&tmem_base_sh, 512);
         tmem_relinquish();
     }
-    if (warp >= 2 && warp < 6) {
-        // One warpgroup writes the constant MMA operands (and makes them
-        // visible to the tensor core: the proxy fence is costly per warp).
-        // Unswizzled K-major [rows][16] bf16 layout: row r, K block kb at
-        // (r / 8) * 256 + kb * 128 + (r % 8) * 16.  The ones matrix has 1.0 in
-        // K elements 0..2 of every row; the bias tiles start all zero and the
-        // producer later writes only K elements 0..2 of each row.
-        const int tid = threadIdx.x - 64;
-        for (int i = tid; i < C::ONES_BYTES / 16; i += 128) {
-            const bool first_block = ((i >> 3) & 1) == 0;   // 16-byte units: 8 rows per K block
-            *reinterpret_cast<uint4 *>(sOnes + i * 16) =
-                first_block ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int st = 0; st < C::NSTAGE; ++st)
-            for (int i = tid; i < 2 * C::BIAS_BYTES / 16; i += 128)
-                *reinterpret_cast<uint4 *>(sQ + st * C::STAGE_BYTES + C::BIAS_T + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_smem();
-    }
+    static_assert(C::LSE_TAB, "the one-item kernel reads the log-sum-exps from tables (no MMA operands to set up)");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -611,16 +619,15 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                     tma_load_3d(st + C::QT_BYTES + b * C::QBLK, &mQs, &bar_qfull[s], b * 64, q0, bh, mdQs, p.st.word);
             }
             float *ktab = reinterpret_cast<float *>(st + C::GK), *gtab = ktab + C::BM;
+            float *ltab = gtab + C::BM, *stab = ltab + C::BM;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int q = lane + 32 * h;
                 ktab[q] = c0[h].w * kLog2eF;
                 gtab[q] = c0[h].z;
-                const uint32_t row = (uint32_t)(q >> 3) * 256u + (uint32_t)(q & 7) * 16u;
-                *reinterpret_cast<uint2 *>(st + C::BIAS_T + row) = split3_bf16(-c0[h].x * p.inv_scale_t);
-                *reinterpret_cast<uint2 *>(st + C::BIAS_S + row) = split3_bf16(-c0[h].y * p.inv_scale_s);
+                ltab[q] = -c0[h].x * kLog2eF;
+                stab[q] = -c0[h].y * kLog2eF;
             }
-            fence_proxy_async_smem();          // the bias rows are read by the tensor core
             mbar_arrive(&bar_qfull[s]);
             issued = t + 1;
         }
@@ -638,8 +645,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
         const uint64_t dKt = sw128_desc(smem_u32(sKt), 16, 1024), dKs = sw128_desc(smem_u32(sKs), 16, 1024);
         const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);          // K-major view of a stage
         const uint64_t dQ0mn = sw128_desc(smem_u32(sQ), C::QBLK, 1024);   // MN-major view of a stage
-        const uint64_t dOnes = plain_desc(smem_u32(sOnes), 128, 256);
-        const uint64_t dBias0 = plain_desc(smem_u32(sQ + C::BIAS_T), 128, 256);
         const bool leader = elect_one();
         const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
         {
@@ -650,7 +655,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                 if (!mbar_wait(&bar_qfull[s], n & 1, p.st, abort_v, 12)) return false;
                 tc_fence_after();
                 const uint64_t dQs = desc_add(dQ0, s * C::STAGE_BYTES + C::QT_BYTES);
-                const uint64_t dBs = desc_add(dBias0, s * C::STAGE_BYTES + C::BIAS_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DS / 16; ++kk) {
                     const uint64_t b = desc_add(dQs, (kk >> 2) * C::QBLK + (kk & 3) * 32);
@@ -660,14 +664,12 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                         mma_bf16_ss(tmem + buf * 128 + 64, desc_add(dKs, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
                                     C::IDESC_S, kk > 0);
                 }
-                mma_bf16_ss(tmem + buf * 128 + 64, dOnes, dBs, C::IDESC_S, 1);
                 return true;
             };
             // Teacher S^T (plus bias) into columns [0, 64), then signal the tile.
             auto issue_st = [&](int t) {
                 const int s = t % C::NSTAGE, buf = t & 1;
                 const uint64_t dQt = desc_add(dQ0, s * C::STAGE_BYTES);
-                const uint64_t dBt = desc_add(dBias0, s * C::STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DT / 16; ++kk) {
                     const uint64_t b = desc_add(dQt, (kk >> 2) * C::QBLK + (kk & 3) * 32);
@@ -677,7 +679,6 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
                         mma_bf16_ss(tmem + buf * 128, desc_add(dKt, (kk >> 2) * C::KBLK + (kk & 3) * 32), b,
                                     C::IDESC_S, kk > 0);
                 }
-                mma_bf16_ss(tmem + buf * 128, dOnes, dBt, C::IDESC_S, 1);
                 mma_commit(&bar_sfull[buf]);
             };
             bool ok = true;
@@ -758,21 +759,25 @@ __global__ void __launch_bounds__(DkvCfg<DT, DS, TEACHER>::THREADS, 1)
             }
             tc_fence_after();
             const float *ktab = reinterpret_cast<const float *>(sQ + s * C::STAGE_BYTES + C::GK) + half * CW;
-            const float *gtab = ktab + C::BM;
+            const float *gtab = ktab + C::BM, *ltab = gtab + C::BM, *stab = ltab + C::BM;
             const int qmin = gk - off - q0;        // first visible query column (causal)
             const uint32_t col = lane_base + buf * 128 + half * CW;   // this warpgroup's chunk
             const bool masked = p.causal && (k0 + C::BN - 1 > q0 + half * CW + off);
             const NamedRel rel{ssid};
             if (masked) {
                 if (p.dkl)
-                    dkv_chunk<TEACHER, true, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW, rel,
-                                                       kNbCount);
+                    dkv_chunk<TEACHER, true, true, CW, kBwdPiece, NamedRel, true>(
+                        col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, qmin - half * CW, rel, kNbCount, ltab, stab);
                 else
-                    dkv_chunk<TEACHER, true, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW, rel,
-                                                        kNbCount);
+                    dkv_chunk<TEACHER, true, false, CW, kBwdPiece, NamedRel, true>(
+                        col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, qmin - half * CW, rel, kNbCount, ltab, stab);
             } else {
-                if (p.dkl) dkv_chunk<TEACHER, false, true, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, rel, kNbCount);
-                else dkv_chunk<TEACHER, false, false, CW>(col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, rel, kNbCount);
+                if (p.dkl)
+                    dkv_chunk<TEACHER, false, true, CW, kBwdPiece, NamedRel, true>(
+                        col, col + 64, p.ct, p.cs, ktab, gtab, 0.f, 0, rel, kNbCount, ltab, stab);
+                else
+                    dkv_chunk<TEACHER, false, false, CW, kBwdPiece, NamedRel, true>(
+                        col, col + 64, p.ct, p.cs, ktab, gtab, g_uni, 0, rel, kNbCount, ltab, stab);
             }
             tmem_st_wait();
             tc_fence_before();
