@@ -17,4 +17,6 @@ def test_the_draws_cover_the_kernel_forms():
     assert any(w.kv_lens for w in ws)
     assert any(w.H_kt < w.H or w.H_ks < w.H for w in ws)
     assert any(w.N_Q < w.N_K for w in ws) and any(w.N_Q > w.N_K for w in ws)
+    assert not any(w.causal and w.N_Q > w.N_K for w in ws)
+    assert any(w.student == "noise" for w in ws) and any(w.student == "independent" for w in ws)
     assert any(w.N_K <= 64 for w in ws) and any(w.N_K > 512 for w in ws)

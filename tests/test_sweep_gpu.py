@@ -3,8 +3,8 @@
 The other GPU tests pick their shapes by hand (tile edges, the five workloads,
 the variants).  This one draws 36 problems from a fixed seed across everything
 the entry points accept at once: batch and head counts, query and key lengths
-from 1 to a few tiles past a multiple of the tile sizes, N_Q < N_K and N_Q >
-N_K, both head dimensions for either model, causal or not, teacher gradients
+from 1 to a few tiles past a multiple of the tile sizes, N_Q < N_K and (not
+causal) N_Q > N_K, both head dimensions for either model, causal or not, teacher gradients
 or not, grouped key heads, padding lengths and a per-row upstream gradient.
 Every draw runs the forward and the full backward through the binding and is
 compared element by element with the oracle (per-row KL and log-sum-exps,
@@ -36,12 +36,17 @@ def draw(i):
     N_Q = r.choice(lengths)
     N_K = r.choice(lengths + [640, 1000])
     causal = r.random() < 0.5
+    if causal and N_Q > N_K:            # the entry points reject it (rows with no key)
+        N_Q, N_K = N_K, N_Q
     kv = ()
     if r.random() < 0.3:
         kv = tuple(r.choice([0, 1, N_K // 2, N_K - 1, N_K]) for _ in range(B))
-    return inputs.custom(f"sweep{i}", B=B, H=H, N_Q=N_Q, N_K=N_K, d_t=r.choice([64, 128]),
-                         d_s=r.choice([64, 128]), causal=causal, student=r.choice(["noise", "independent"]),
-                         teacher_grads=r.random() < 0.5, seed=7000 + i, h_kt=H // group_t, h_ks=H // group_s,
+    d_t, d_s = r.choice([64, 128]), r.choice([64, 128])
+    h_kt, h_ks = H // group_t, H // group_s
+    # a student drawn as the teacher plus noise needs the teacher's shapes
+    student = r.choice(["noise", "independent"]) if (d_t, h_kt) == (d_s, h_ks) else "independent"
+    return inputs.custom(f"sweep{i}", B=B, H=H, N_Q=N_Q, N_K=N_K, d_t=d_t, d_s=d_s, causal=causal,
+                         student=student, teacher_grads=r.random() < 0.5, seed=7000 + i, h_kt=h_kt, h_ks=h_ks,
                          kv_lens=kv), r.random() < 0.5
 
 
