@@ -226,10 +226,12 @@ __device__ __forceinline__ void dq_chunk(uint32_t at, uint32_t as, float ct, flo
     store_ds<TEACHER, CWID>(at, ps, pt);
 }
 
-// Key-owner chunk (thread = key row; the logits already carry -LSE / scale, so
-// only KL log2(e) per query column comes from shared memory, `ktab`, and g
-// too when it varies per row (G_ROW: `gtab`; otherwise g is uniform and the
-// caller applies it to the accumulated dK instead).
+// Key-owner chunk (thread = key row).  The per-query values come from
+// shared-memory tables: KL log2(e) (`ktab`), g when it varies per row (G_ROW:
+// `gtab`; otherwise g is uniform and the caller applies it to the accumulated
+// dK instead) and, with LTAB, -LSE_t log2(e) and -LSE_s log2(e) (`ltab`,
+// `stab`), folded into the first fused multiply-add; without LTAB the logits
+// already carry -LSE / scale (a rank-1 bias MMA added it).
 // Every thread of the warp reads the same four floats with one 16-byte
 // broadcast load per four columns (a quarter of the load instructions of
 // 4-byte loads, for the same shared-memory wavefronts per value; measured
